@@ -1,0 +1,372 @@
+#!/usr/bin/env python
+"""Benchmark of the RainFusion2.0 block-sparse attention path on B200.
+
+One step = the whole hot path on one Wan2.2-shaped 720p attention call (B=1, 40 heads,
+21x45x80 latent tokens, head_dim 128, window 2x8x8, 80% sparsity, first-frame sink):
+3D-window permute of Q/K/V -> block-mean pooling -> pooled scores -> sink + top-k ->
+block-sparse attention -> inverse permute, each through the library's C ABI.
+
+Prints one JSON line (rank 0).  `value` is dense-equivalent TFLOP/s (4*B*heads*N^2*D
+over the unpadded N, per call) summed over ranks; `ms_per_step` is ms per call.
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same call.
+Multi-GPU (torchrun): every rank runs its own call (independent replicas, weak scaling);
+the only collectives are the barrier and the max over ranks of the timings.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "wan720p"
+
+
+def _args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="rf2", choices=["rf2", "reference"])
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--sparsity", type=float, default=None)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    return p.parse_args()
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def _geometry_numbers(g, kept):
+    dense = 4.0 * g.B * g.heads * float(g.N) ** 2 * g.D
+    kept_flop = 4.0 * g.B * g.heads * g.Nb * kept * g.blk * g.blk * g.D
+    mask_bytes = 2.0 * g.B * g.Npad * g.heads * g.D * 2  # padded Q and K read once
+    permute_bytes = 3.0 * g.B * (g.N + g.Npad) * g.heads * g.D * 2
+    unpermute_bytes = 1.0 * g.B * (g.N + g.Npad) * g.heads * g.D * 2
+    return dense, kept_flop, mask_bytes, permute_bytes, unpermute_bytes
+
+
+def _traffic_from_profile(kernel_src_sha):
+    """DRAM bytes per launch of the attention kernel from the committed ncu summary, if
+    it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "sparse_attn_wan720p.md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    m_sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", txt)
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    if not m_sha or not m_b or m_sha.group(1) != kernel_src_sha:
+        return None
+    return float(m_b.group(1))
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for fn in ("attn.cu", "sm100_ptx.cuh"):
+        with open(os.path.join(ROOT, "image_diffusion_dits_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = [ln.split(",") for ln in (self.out or "").strip().splitlines() if ln.count(",") >= 8]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+def run_cpu_baseline(wl, sparsity, seconds, rows_cap=64):
+    """The fp64 oracle on a bounded sample of the same call: its mask stage on the full
+    call is skipped (attention dominates); attention is timed on sampled (head, query
+    block) rows and scaled to the full call."""
+    import numpy as np
+    import torch
+
+    import oracle as O
+    from rf2_inputs import bf16_bits_to_f64, gen_tensor
+
+    og = O.geom(**wl.geom())
+    cores = len(os.sched_getaffinity(0))
+    torch.set_num_threads(cores)
+    # a single head of the call is generated (the oracle's cost is per head)
+    one = dict(wl.geom())
+    one["heads"] = 1
+    g1 = O.geom(**one)
+    q, k, v = (bf16_bits_to_f64(gen_tensor(1, wl.T, wl.H, wl.W, 1, wl.D, 1000 * wl.cfg + i)) for i in range(3))
+    qp, kp, vp = (O.permute(a, g1) for a in (q, k, v))
+    t0 = time.perf_counter()
+    sel = O.predict_mask(qp, kp, g1, sparsity, wl.sink)
+    t_mask_head = time.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    order = rng.permutation(g1.Nb)
+    sc = 1.0 / math.sqrt(wl.D)
+    done = 0
+    t0 = time.perf_counter()
+    while done < min(rows_cap, g1.Nb) and time.perf_counter() - t0 < seconds:
+        i = int(order[done])
+        O.attention_block(qp, kp, vp, g1, 0, 0, i, sel.idx[0, 0, i], sc)
+        done += 1
+    t_attn = time.perf_counter() - t0
+    per_row = t_attn / done
+    call_s = (per_row * og.Nb + t_mask_head) * og.heads * og.B
+    return {"call_s": call_s, "cores": cores, "rows": done, "per_row_s": per_row,
+            "mask_head_s": t_mask_head}
+
+
+def main():
+    a = _args()
+    import torch
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from rf2_inputs import WORKLOADS
+
+    wl = WORKLOADS[a.workload]
+    sparsity = wl.sparsity if a.sparsity is None else a.sparsity
+    metric = "ms/call and dense-equiv TFLOP/s at 80% sparsity, Wan-720p-shaped attention"
+    unit = "dense-equiv TFLOP/s"
+
+    if a.impl == "reference":
+        if rank != 0:
+            return 0
+        import oracle as O
+
+        g = O.geom(**wl.geom())
+        kept = O.kept_count(g, sparsity, wl.sink)
+        dense = _geometry_numbers(g, kept)[0]
+        per_step = []
+        cb = None
+        for step in range(a.warmup + a.steps):
+            cb = run_cpu_baseline(wl, sparsity, seconds=max(2.0, a.cpu_seconds / max(a.steps, 1)), rows_cap=8)
+            if step >= a.warmup:
+                per_step.append(cb["call_s"])
+        call_s = statistics.mean(per_step)
+        val = dense / call_s / 1e12 * world
+        line = {"impl": "reference", "metric": metric, "value": val, "unit": unit, "n_gpus": world,
+                "steps": a.steps, "warmup": a.warmup, "ms_per_step": call_s * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": f"{wl.name}: B={wl.B} heads={wl.heads} grid={wl.T}x{wl.H}x{wl.W} "
+                                       f"D={wl.D} window={wl.wt}x{wl.wh}x{wl.ww} sparsity={sparsity} sink={wl.sink}"},
+                "cpu_baseline": {"value": val, "unit": unit, "cores": cb["cores"], "kind": "oracle",
+                                 "sample": f"per step: attention of {cb['rows']} sampled query blocks of one "
+                                           f"head plus that head's mask stage, scaled to all "
+                                           f"{wl.heads} heads x {g.Nb} query blocks"},
+                "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import image_diffusion_dits_b200 as rf2
+    from rf2_inputs import gen_tensor_torch
+
+    if world > 1:
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    g = rf2.Geometry(**wl.geom())
+    kept = rf2.kept_count(g, sparsity, wl.sink)
+    dense, kept_flop, mask_bytes, perm_bytes, unperm_bytes = _geometry_numbers(g, kept)
+
+    seed0 = 1000 * wl.cfg + 100 * rank
+    q, k, v = (gen_tensor_torch(g.B, g.T, g.H, g.W, g.heads, g.D, seed0 + i, dev) for i in range(3))
+    shp = (g.B, g.Npad, g.heads, g.D)
+    qp, kp, vp, op = (torch.empty(shp, dtype=torch.bfloat16, device=dev) for _ in range(4))
+    o = torch.empty_like(q)
+    idx = torch.empty((g.B, g.heads, g.Nb, kept), dtype=torch.int32, device=dev)
+    cnt = torch.empty((g.B, g.heads, g.Nb), dtype=torch.int32, device=dev)
+    mws = torch.empty(rf2.workspace_size(g, sparsity, wl.sink, attention=False), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    n_seg = 4
+    evs = None
+
+    def step(record):
+        if record:
+            record[0].record(stream)
+        rf2.permute(q, g, out=qp)
+        rf2.permute(k, g, out=kp)
+        rf2.permute(v, g, out=vp)
+        if record:
+            record[1].record(stream)
+        rf2.predict_mask(qp, kp, g, sparsity, wl.sink, kmax=kept, ws=mws, out=(idx, cnt))
+        if record:
+            record[2].record(stream)
+        rf2.sparse_attn(qp, kp, vp, idx, cnt, g, out=op, status=status)
+        if record:
+            record[3].record(stream)
+        rf2.unpermute(op, g, out=o)
+        if record:
+            record[4].record(stream)
+
+    launches_per_step = 3 + 3 + 1 + 1
+    for _ in range(a.warmup):
+        step(None)
+    torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} after warm-up")
+
+    seg_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_seg + 1)] for _ in range(a.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        start.record(stream)
+        for s in range(a.steps):
+            step(seg_ev[s])
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = start.elapsed_time(end)
+    seg_ms = [sum(seg_ev[s][i].elapsed_time(seg_ev[s][i + 1]) for s in range(a.steps)) / a.steps
+              for i in range(n_seg)]
+    if world > 1:
+        t = torch.tensor([total_ms] + seg_ms, dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms, seg_ms = float(t[0]), [float(x) for x in t[1:]]
+    ms_per_step = total_ms / a.steps
+    value = dense * world / (ms_per_step * 1e-3) / 1e12
+    peaks = _peaks()
+
+    # end to end through the public fused call: pinned host inputs in, host output back
+    e2e = None
+    if not a.no_e2e:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        ws = torch.empty(rf2.workspace_size(g, sparsity, wl.sink), dtype=torch.uint8, device=dev)
+        dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+        for it in range(a.warmup + a.steps):
+            if it == a.warmup:
+                if world > 1:
+                    torch.distributed.barrier()
+                torch.cuda.synchronize(dev)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            rf2.attention(dq, dk, dv, g, sparsity, wl.sink, ws=ws, out=o)
+            ho.copy_(o, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1) / a.steps
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t[0])
+        e2e = {"value": dense * world / (e2e_ms * 1e-3) / 1e12, "unit": unit, "ms_per_call": e2e_ms,
+               "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": o.numel() * 2}
+        del ws, dq, dk, dv
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        cb = run_cpu_baseline(wl, sparsity, a.cpu_seconds)
+        cpu = {"value": dense / cb["call_s"] / 1e12, "unit": unit, "cores": cb["cores"], "kind": "oracle",
+               "ms_per_call": cb["call_s"] * 1e3,
+               "sample": f"attention of {cb['rows']} sampled query blocks of one head (fp64 NumPy) plus that "
+                         f"head's mask stage, scaled to {wl.heads} heads x {g.Nb} query blocks"}
+
+    attn_ms = seg_ms[2]
+    achieved = kept_flop / (attn_ms * 1e-3) / 1e12
+    sha = kernel_source_sha()
+    traffic = _traffic_from_profile(sha)
+    mask_gbs = mask_bytes / (seg_ms[1] * 1e-3) / 1e9
+    line = {
+        "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{wl.name}: B={wl.B} heads={wl.heads} grid={wl.T}x{wl.H}x{wl.W} "
+                               f"(padded {g.Npad} tokens) D={wl.D} window={wl.wt}x{wl.wh}x{wl.ww} "
+                               f"sparsity={sparsity} sink={wl.sink} kept={kept}/{g.Nb}",
+                   "l2": "inputs larger than L2 (774 MB per tensor); no flush",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                     "kernel": "sparse_attn_kernel<128,128>", "peak_source": peaks["source"] + " burst",
+                     "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
+                                           if peaks.get("bf16_tflops_sustained") else None),
+                     "kernel_source_sha": sha},
+        "stages_ms": {"permute_qkv": seg_ms[0], "predict_mask": seg_ms[1], "sparse_attn": seg_ms[2],
+                      "unpermute": seg_ms[3]},
+        "mask_stage": {"ms": seg_ms[1], "GB/s": mask_gbs, "frac_hbm": mask_gbs / peaks["hbm_gbs"]},
+        "permute_GB/s": perm_bytes / (seg_ms[0] * 1e-3) / 1e9,
+        "clocks": clk.summary(),
+        "gpu_launches": launches_per_step * a.steps,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

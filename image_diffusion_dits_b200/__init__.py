@@ -1,0 +1,201 @@
+"""B200 (sm_100a) RainFusion2.0 block-sparse attention: Python binding of librf2.so.
+
+Every function here marshals torch tensors (device memory, current stream) into the C ABI
+of include/rf2.h; all computation runs in the library's CUDA kernels.  There is no CPU
+path: the functions raise if the library is missing or a tensor is not on a CUDA device.
+
+Layouts: model-order Q/K/V/O are [B, T*H*W, heads, D] bf16 (raster token order);
+permuted tensors are [B, Npad, heads, D] bf16 in 3D-window order.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+from typing import Optional, Tuple
+
+import torch
+
+from . import _lib
+from ._lib import RF2_CHECKED, RF2_SINK_ADDITIVE, Rf2Geom
+
+__all__ = [
+    "Geometry", "Rf2Error", "permute", "unpermute", "kept_count", "workspace_size",
+    "predict_mask", "sparse_attn", "attention", "library",
+]
+
+
+class Rf2Error(RuntimeError):
+    def __init__(self, code: int, where: str):
+        msg = _lib.load().rf2_status_string(code).decode()
+        super().__init__(f"{where}: {msg} (status {code})")
+        self.code = code
+
+
+@dataclasses.dataclass(frozen=True)
+class Geometry:
+    """Shape of one attention call: batch, heads, token grid, head_dim, 3D window."""
+
+    B: int
+    heads: int
+    T: int
+    H: int
+    W: int
+    D: int
+    wt: int
+    wh: int
+    ww: int
+
+    @property
+    def N(self) -> int:
+        return self.T * self.H * self.W
+
+    @property
+    def blk(self) -> int:
+        return self.wt * self.wh * self.ww
+
+    @property
+    def Nb(self) -> int:
+        c = lambda a, b: -(-a // b)
+        return c(self.T, self.wt) * c(self.H, self.wh) * c(self.W, self.ww)
+
+    @property
+    def Npad(self) -> int:
+        return self.Nb * self.blk
+
+    def c(self) -> Rf2Geom:
+        return Rf2Geom(self.B, self.heads, self.T, self.H, self.W, self.D, self.wt, self.wh, self.ww)
+
+
+def library() -> ctypes.CDLL:
+    return _lib.load()
+
+
+def _check(code: int, where: str) -> None:
+    if code != 0:
+        raise Rf2Error(code, where)
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _cuda_bf16(t: torch.Tensor, name: str, shape) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+    if t.dtype != torch.bfloat16 or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected contiguous bf16 {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+
+
+def _flags(additive: bool, checked: bool) -> int:
+    return (RF2_SINK_ADDITIVE if additive else 0) | (RF2_CHECKED if checked else 0)
+
+
+def permute(x: torch.Tensor, g: Geometry, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _cuda_bf16(x, "x", (g.B, g.N, g.heads, g.D))
+    if out is None:
+        out = torch.empty((g.B, g.Npad, g.heads, g.D), dtype=torch.bfloat16, device=x.device)
+    cg = g.c()
+    _check(library().rf2_permute(x.data_ptr(), out.data_ptr(), ctypes.byref(cg), _stream(x)), "rf2_permute")
+    return out
+
+
+def unpermute(xp: torch.Tensor, g: Geometry, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _cuda_bf16(xp, "xp", (g.B, g.Npad, g.heads, g.D))
+    if out is None:
+        out = torch.empty((g.B, g.N, g.heads, g.D), dtype=torch.bfloat16, device=xp.device)
+    cg = g.c()
+    _check(library().rf2_unpermute(xp.data_ptr(), out.data_ptr(), ctypes.byref(cg), _stream(xp)),
+           "rf2_unpermute")
+    return out
+
+
+def kept_count(g: Geometry, sparsity: float, sink: bool, additive: bool = False) -> int:
+    cg = g.c()
+    k = library().rf2_kept_count(ctypes.byref(cg), float(sparsity), int(sink), _flags(additive, False))
+    if k < 0:
+        raise Rf2Error(-k, "rf2_kept_count")
+    return k
+
+
+def workspace_size(g: Geometry, sparsity: float, sink: bool, additive: bool = False,
+                   attention: bool = True) -> int:
+    cg = g.c()
+    n = library().rf2_workspace_size(ctypes.byref(cg), float(sparsity), int(sink),
+                                     _flags(additive, False), int(attention))
+    if n == 0:
+        raise Rf2Error(_lib.RF2_ERR_INVALID_ARG, "rf2_workspace_size")
+    return n
+
+
+def predict_mask(qp: torch.Tensor, kp: torch.Tensor, g: Geometry, sparsity: float, sink: bool,
+                 additive: bool = False, kmax: Optional[int] = None, checked: bool = False,
+                 ws: Optional[torch.Tensor] = None,
+                 out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Kept block lists idx [B, heads, Nb, kmax] (ascending, -1 padded) and counts."""
+    _cuda_bf16(qp, "qp", (g.B, g.Npad, g.heads, g.D))
+    _cuda_bf16(kp, "kp", (g.B, g.Npad, g.heads, g.D))
+    k = kept_count(g, sparsity, sink, additive) if kmax is None else kmax
+    if out is None:
+        idx = torch.empty((g.B, g.heads, g.Nb, k), dtype=torch.int32, device=qp.device)
+        cnt = torch.empty((g.B, g.heads, g.Nb), dtype=torch.int32, device=qp.device)
+    else:
+        idx, cnt = out
+        if idx.dtype != torch.int32 or cnt.dtype != torch.int32 or idx.shape[-1] != k:
+            raise ValueError("out must be int32 (idx [B, heads, Nb, kmax], cnt [B, heads, Nb])")
+    nbytes = workspace_size(g, sparsity, sink, additive, attention=False)
+    if ws is None:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=qp.device)
+    cg = g.c()
+    _check(library().rf2_predict_mask(qp.data_ptr(), kp.data_ptr(), ctypes.byref(cg), float(sparsity),
+                                      int(sink), _flags(additive, checked), idx.data_ptr(), cnt.data_ptr(),
+                                      k, ws.data_ptr(), ws.numel(), _stream(qp)), "rf2_predict_mask")
+    return idx, cnt
+
+
+def sparse_attn(qp: torch.Tensor, kp: torch.Tensor, vp: torch.Tensor, idx: torch.Tensor,
+                cnt: torch.Tensor, g: Geometry, scale: float = 0.0, checked: bool = False,
+                out: Optional[torch.Tensor] = None,
+                status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    for t, n in ((qp, "qp"), (kp, "kp"), (vp, "vp")):
+        _cuda_bf16(t, n, (g.B, g.Npad, g.heads, g.D))
+    if idx.dtype != torch.int32 or cnt.dtype != torch.int32 or not idx.is_contiguous():
+        raise ValueError("idx and cnt must be contiguous int32")
+    if out is None:
+        out = torch.empty_like(qp)
+    if status is None and checked:
+        status = torch.zeros(1, dtype=torch.int32, device=qp.device)
+    cg = g.c()
+    _check(library().rf2_sparse_attn(qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), idx.data_ptr(),
+                                     cnt.data_ptr(), idx.shape[-1], ctypes.byref(cg), float(scale),
+                                     out.data_ptr(), 0 if status is None else status.data_ptr(),
+                                     _flags(False, checked), _stream(qp)), "rf2_sparse_attn")
+    return out
+
+
+def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Geometry, sparsity: float,
+              sink: bool = True, scale: float = 0.0, additive: bool = False,
+              return_idx: bool = False, checked: bool = False,
+              ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None):
+    """The whole RF2 path: permute -> mask -> block-sparse attention -> unpermute."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _cuda_bf16(t, n, (g.B, g.N, g.heads, g.D))
+    nbytes = workspace_size(g, sparsity, sink, additive, attention=True)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    idx = None
+    if return_idx:
+        kk = kept_count(g, sparsity, sink, additive)
+        idx = torch.empty((g.B, g.heads, g.Nb, kk), dtype=torch.int32, device=q.device)
+    cg = g.c()
+    _check(library().rf2_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(cg),
+                                   float(sparsity), int(sink), float(scale), out.data_ptr(),
+                                   0 if idx is None else idx.data_ptr(), ws.data_ptr(), ws.numel(),
+                                   _flags(additive, checked), _stream(q)), "rf2_attention")
+    return (out, idx) if return_idx else out
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)

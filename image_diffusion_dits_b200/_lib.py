@@ -1,0 +1,75 @@
+"""ctypes declarations of librf2.so (the C ABI in include/rf2.h).  Argument marshalling only."""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "librf2.so")
+
+RF2_OK = 0
+RF2_ERR_INVALID_ARG = 1
+RF2_ERR_UNSUPPORTED = 2
+RF2_ERR_ALIGNMENT = 3
+RF2_ERR_WORKSPACE = 4
+RF2_ERR_BAD_INDEX = 5
+RF2_ERR_TIMEOUT = 6
+RF2_ERR_CUDA = 7
+
+RF2_SINK_ADDITIVE = 1
+RF2_CHECKED = 2
+
+# Every symbol include/rf2.h declares.
+EXPORTS = (
+    "rf2_permute",
+    "rf2_unpermute",
+    "rf2_kept_count",
+    "rf2_workspace_size",
+    "rf2_predict_mask",
+    "rf2_sparse_attn",
+    "rf2_attention",
+    "rf2_status_string",
+)
+
+
+class Rf2Geom(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("B", "heads", "T", "H", "W", "D", "wt", "wh", "ww")]
+
+
+_vp = ctypes.c_void_p
+_i32p = ctypes.c_void_p  # device int32* passed as a raw address
+_gp = ctypes.POINTER(Rf2Geom)
+
+_SIGS = {
+    "rf2_permute": (ctypes.c_int, [_vp, _vp, _gp, _vp]),
+    "rf2_unpermute": (ctypes.c_int, [_vp, _vp, _gp, _vp]),
+    "rf2_kept_count": (ctypes.c_int, [_gp, ctypes.c_double, ctypes.c_int, ctypes.c_uint]),
+    "rf2_workspace_size": (ctypes.c_size_t, [_gp, ctypes.c_double, ctypes.c_int, ctypes.c_uint,
+                                             ctypes.c_int]),
+    "rf2_predict_mask": (ctypes.c_int, [_vp, _vp, _gp, ctypes.c_double, ctypes.c_int, ctypes.c_uint,
+                                        _i32p, _i32p, ctypes.c_int, _vp, ctypes.c_size_t, _vp]),
+    "rf2_sparse_attn": (ctypes.c_int, [_vp, _vp, _vp, _i32p, _i32p, ctypes.c_int, _gp, ctypes.c_float,
+                                       _vp, _i32p, ctypes.c_uint, _vp]),
+    "rf2_attention": (ctypes.c_int, [_vp, _vp, _vp, _gp, ctypes.c_double, ctypes.c_int, ctypes.c_float,
+                                     _vp, _i32p, _vp, ctypes.c_size_t, ctypes.c_uint, _vp]),
+    "rf2_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+}
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load librf2.so (once).  Raises if it has not been built: there is no fallback."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise ImportError(
+                f"librf2.so not found at {path}; build it with "
+                "`python -m image_diffusion_dits_b200.build` (needs nvcc)")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib

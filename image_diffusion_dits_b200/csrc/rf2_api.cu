@@ -1,0 +1,278 @@
+// C ABI of the block-sparse attention library: argument validation, workspace layout,
+// and the launch sequence of each entry point.  Every compute step runs in the CUDA
+// kernels of permute.cu, mask.cu and attn.cu.
+#include <math.h>
+#include <stdio.h>
+#include <stdlib.h>
+
+#include "rf2_common.cuh"
+
+using rf2::Geo;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_geom(const rf2_geom* g) {
+  if (g == nullptr) return RF2_ERR_INVALID_ARG;
+  if (g->B < 1 || g->heads < 1 || g->T < 1 || g->H < 1 || g->W < 1 || g->wt < 1 || g->wh < 1 ||
+      g->ww < 1 || g->D < 1)
+    return RF2_ERR_INVALID_ARG;
+  if (g->D != 64 && g->D != 128) return RF2_ERR_UNSUPPORTED;
+  const long long blk = (long long)g->wt * g->wh * g->ww;
+  if (blk != 64 && blk != 128) return RF2_ERR_UNSUPPORTED;
+  Geo o = rf2::make_geo(*g);
+  if (o.Nb > 1024) return RF2_ERR_UNSUPPORTED;                  // kept lists live in smem
+  if ((long long)o.B * o.Npad >= (1ll << 31)) return RF2_ERR_UNSUPPORTED;  // TMA coordinates
+  return RF2_OK;
+}
+
+int nsink_of(const Geo& g, int sink) { return sink ? g.nbh * g.nbw : 0; }
+
+// Kept blocks per row (both sides of the sink reading).  Every block holds at least one
+// real token (padding is less than one window per axis), so all Nb blocks are valid.
+int kept_of(const Geo& g, double sparsity, int sink, unsigned flags) {
+  const int nv = g.Nb;
+  const int ns = nsink_of(g, sink);
+  if (flags & RF2_SINK_ADDITIVE) {
+    long long extra = (long long)ceil((1.0 - sparsity) * (double)(nv - ns) - 1e-6);
+    if (extra < 0) extra = 0;
+    if (extra > nv - ns) extra = nv - ns;
+    return ns + (int)extra;
+  }
+  long long k = (long long)ceil((1.0 - sparsity) * (double)nv - 1e-6);
+  if (k < 1) k = 1;
+  if (k > nv) k = nv;
+  return (int)(k > ns ? k : ns);
+}
+
+struct MaskWs {
+  int32_t* status;
+  float* qbar;
+  float* kbar;
+  float* scores;
+  size_t bytes;
+};
+
+MaskWs mask_ws_layout(const Geo& g, uint8_t* base) {
+  MaskWs w;
+  size_t off = 0;
+  w.status = reinterpret_cast<int32_t*>(base + off);
+  off += kAlign;
+  const size_t means = (size_t)g.B * g.heads * g.Nb * g.D * sizeof(float);
+  w.qbar = reinterpret_cast<float*>(base + off);
+  off += align_up(means);
+  w.kbar = reinterpret_cast<float*>(base + off);
+  off += align_up(means);
+  w.scores = reinterpret_cast<float*>(base + off);
+  off += align_up((size_t)g.B * g.heads * g.Nb * g.Nb * sizeof(float));
+  w.bytes = off;
+  return w;
+}
+
+struct AttnWs {
+  MaskWs mask;
+  void *qp, *kp, *vp, *op;
+  int32_t *idx, *cnt;
+  size_t bytes;
+};
+
+AttnWs attn_ws_layout(const Geo& g, int kept, uint8_t* base) {
+  AttnWs w;
+  w.mask = mask_ws_layout(g, base);
+  size_t off = w.mask.bytes;
+  const size_t t = align_up((size_t)g.B * g.Npad * g.heads * g.D * 2);
+  w.qp = base + off; off += t;
+  w.kp = base + off; off += t;
+  w.vp = base + off; off += t;
+  w.op = base + off; off += t;
+  w.idx = reinterpret_cast<int32_t*>(base + off);
+  off += align_up((size_t)g.B * g.heads * g.Nb * kept * sizeof(int32_t));
+  w.cnt = reinterpret_cast<int32_t*>(base + off);
+  off += align_up((size_t)g.B * g.heads * g.Nb * sizeof(int32_t));
+  w.bytes = off;
+  return w;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? RF2_OK : RF2_ERR_CUDA; }
+
+bool log_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* s = getenv("RF2_LOG");
+    v = (s != nullptr && s[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
+
+void log_geo(const char* what, const Geo& g, int kept) {
+  if (!log_enabled()) return;
+  fprintf(stderr,
+          "[rf2] %s B=%d heads=%d grid=%dx%dx%d D=%d window=%dx%dx%d Nb=%d blk=%d Npad=%lld "
+          "kept=%d\n",
+          what, g.B, g.heads, g.T, g.H, g.W, g.D, g.wt, g.wh, g.ww, g.Nb, g.blk, g.Npad, kept);
+}
+
+// In checked mode: wait for the stream and return the device status word.
+int finish_checked(unsigned flags, const int32_t* status_dev, cudaStream_t s) {
+  if (!(flags & RF2_CHECKED)) return RF2_OK;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return RF2_ERR_CUDA;
+  if (status_dev == nullptr) return RF2_OK;
+  int32_t st = 0;
+  e = cudaMemcpyAsync(&st, status_dev, sizeof(st), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return RF2_ERR_CUDA;
+  return st;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* rf2_status_string(int status) {
+  switch (status) {
+    case RF2_OK: return "ok";
+    case RF2_ERR_INVALID_ARG: return "invalid argument";
+    case RF2_ERR_UNSUPPORTED: return "unsupported shape (D and block size must be 64 or 128, Nb <= 1024)";
+    case RF2_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case RF2_ERR_WORKSPACE: return "workspace missing or too small";
+    case RF2_ERR_BAD_INDEX: return "kept block index out of range";
+    case RF2_ERR_TIMEOUT: return "device wait timed out";
+    case RF2_ERR_CUDA: return "CUDA error";
+    default: return "unknown status";
+  }
+}
+
+int rf2_permute(const void* x, void* xp, const rf2_geom* g, void* stream) {
+  int st = check_geom(g);
+  if (st != RF2_OK) return st;
+  if (x == nullptr || xp == nullptr) return RF2_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xp)) return RF2_ERR_ALIGNMENT;
+  Geo geo = rf2::make_geo(*g);
+  log_geo("permute", geo, 0);
+  return cuda_status(rf2::launch_permute(x, xp, geo, (cudaStream_t)stream));
+}
+
+int rf2_unpermute(const void* xp, void* x, const rf2_geom* g, void* stream) {
+  int st = check_geom(g);
+  if (st != RF2_OK) return st;
+  if (x == nullptr || xp == nullptr) return RF2_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xp)) return RF2_ERR_ALIGNMENT;
+  Geo geo = rf2::make_geo(*g);
+  log_geo("unpermute", geo, 0);
+  return cuda_status(rf2::launch_unpermute(xp, x, geo, (cudaStream_t)stream));
+}
+
+int rf2_kept_count(const rf2_geom* g, double sparsity, int sink, unsigned flags) {
+  int st = check_geom(g);
+  if (st != RF2_OK) return -st;
+  if (!(sparsity >= 0.0 && sparsity <= 1.0)) return -RF2_ERR_INVALID_ARG;
+  return kept_of(rf2::make_geo(*g), sparsity, sink, flags);
+}
+
+size_t rf2_workspace_size(const rf2_geom* g, double sparsity, int sink, unsigned flags,
+                          int attention) {
+  if (check_geom(g) != RF2_OK) return 0;
+  if (!(sparsity >= 0.0 && sparsity <= 1.0)) return 0;
+  Geo geo = rf2::make_geo(*g);
+  if (!attention) return mask_ws_layout(geo, nullptr).bytes;
+  return attn_ws_layout(geo, kept_of(geo, sparsity, sink, flags), nullptr).bytes;
+}
+
+static int predict_mask_impl(const void* qp, const void* kp, const Geo& geo, double sparsity,
+                             int sink, unsigned flags, int32_t* idx, int32_t* cnt, int kmax,
+                             const MaskWs& w, cudaStream_t s) {
+  const int kept = kept_of(geo, sparsity, sink, flags);
+  log_geo("predict_mask", geo, kept);
+  cudaError_t e = rf2::launch_pool(qp, kp, w.qbar, w.kbar, geo, s);
+  if (e == cudaSuccess)
+    e = rf2::launch_scores(w.qbar, w.kbar, w.scores, geo, (float)(1.0 / sqrt((double)geo.D)), s);
+  if (e == cudaSuccess)
+    e = rf2::launch_topk(w.scores, idx, cnt, kmax, kept, nsink_of(geo, sink), geo, s);
+  return cuda_status(e);
+}
+
+int rf2_predict_mask(const void* qp, const void* kp, const rf2_geom* g, double sparsity, int sink,
+                     unsigned flags, int32_t* idx, int32_t* cnt, int kmax, void* ws,
+                     size_t ws_bytes, void* stream) {
+  int st = check_geom(g);
+  if (st != RF2_OK) return st;
+  if (!(sparsity >= 0.0 && sparsity <= 1.0)) return RF2_ERR_INVALID_ARG;
+  if (qp == nullptr || kp == nullptr || idx == nullptr || cnt == nullptr) return RF2_ERR_INVALID_ARG;
+  if (!aligned16(qp) || !aligned16(kp) || !aligned16(idx) || !aligned16(cnt))
+    return RF2_ERR_ALIGNMENT;
+  Geo geo = rf2::make_geo(*g);
+  if (kmax < kept_of(geo, sparsity, sink, flags)) return RF2_ERR_INVALID_ARG;
+  if (ws == nullptr || !aligned16(ws)) return ws == nullptr ? RF2_ERR_WORKSPACE : RF2_ERR_ALIGNMENT;
+  MaskWs w = mask_ws_layout(geo, static_cast<uint8_t*>(ws));
+  if (ws_bytes < w.bytes) return RF2_ERR_WORKSPACE;
+  st = predict_mask_impl(qp, kp, geo, sparsity, sink, flags, idx, cnt, kmax, w,
+                         (cudaStream_t)stream);
+  if (st != RF2_OK) return st;
+  return finish_checked(flags, nullptr, (cudaStream_t)stream);
+}
+
+int rf2_sparse_attn(const void* qp, const void* kp, const void* vp, const int32_t* idx,
+                    const int32_t* cnt, int kmax, const rf2_geom* g, float scale, void* op,
+                    int32_t* status, unsigned flags, void* stream) {
+  int st = check_geom(g);
+  if (st != RF2_OK) return st;
+  if (qp == nullptr || kp == nullptr || vp == nullptr || idx == nullptr || cnt == nullptr ||
+      op == nullptr || kmax < 1 || !isfinite(scale))
+    return RF2_ERR_INVALID_ARG;
+  if (!aligned16(qp) || !aligned16(kp) || !aligned16(vp) || !aligned16(op) ||
+      ((uintptr_t)idx & 3u) || ((uintptr_t)cnt & 3u) || ((uintptr_t)status & 3u))
+    return RF2_ERR_ALIGNMENT;
+  Geo geo = rf2::make_geo(*g);
+  const float sc = scale == 0.f ? (float)(1.0 / sqrt((double)geo.D)) : scale;
+  log_geo("sparse_attn", geo, kmax);
+  cudaError_t e = rf2::launch_sparse_attn(qp, kp, vp, idx, cnt, kmax, geo, sc, op, status,
+                                          (cudaStream_t)stream);
+  if (e == cudaErrorNotSupported) return RF2_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return RF2_ERR_CUDA;
+  return finish_checked(flags, status, (cudaStream_t)stream);
+}
+
+int rf2_attention(const void* q, const void* k, const void* v, const rf2_geom* g, double sparsity,
+                  int sink, float scale, void* o, int32_t* idx_out, void* ws, size_t ws_bytes,
+                  unsigned flags, void* stream) {
+  int st = check_geom(g);
+  if (st != RF2_OK) return st;
+  if (!(sparsity >= 0.0 && sparsity <= 1.0) || !isfinite(scale)) return RF2_ERR_INVALID_ARG;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return RF2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      ((uintptr_t)idx_out & 3u))
+    return RF2_ERR_ALIGNMENT;
+  if (ws == nullptr) return RF2_ERR_WORKSPACE;
+  if (!aligned16(ws)) return RF2_ERR_ALIGNMENT;
+  Geo geo = rf2::make_geo(*g);
+  const int kept = kept_of(geo, sparsity, sink, flags);
+  AttnWs w = attn_ws_layout(geo, kept, static_cast<uint8_t*>(ws));
+  if (ws_bytes < w.bytes) return RF2_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  const float sc = scale == 0.f ? (float)(1.0 / sqrt((double)geo.D)) : scale;
+  log_geo("attention", geo, kept);
+  cudaError_t e = cudaMemsetAsync(w.mask.status, 0, sizeof(int32_t), s);
+  if (e == cudaSuccess) e = rf2::launch_permute(q, w.qp, geo, s);
+  if (e == cudaSuccess) e = rf2::launch_permute(k, w.kp, geo, s);
+  if (e == cudaSuccess) e = rf2::launch_permute(v, w.vp, geo, s);
+  if (e != cudaSuccess) return RF2_ERR_CUDA;
+  st = predict_mask_impl(w.qp, w.kp, geo, sparsity, sink, flags, w.idx, w.cnt, kept, w.mask, s);
+  if (st != RF2_OK) return st;
+  e = rf2::launch_sparse_attn(w.qp, w.kp, w.vp, w.idx, w.cnt, kept, geo, sc, w.op,
+                              w.mask.status, s);
+  if (e == cudaErrorNotSupported) return RF2_ERR_UNSUPPORTED;
+  if (e == cudaSuccess) e = rf2::launch_unpermute(w.op, o, geo, s);
+  if (e == cudaSuccess && idx_out != nullptr)
+    e = cudaMemcpyAsync(idx_out, w.idx, (size_t)geo.B * geo.heads * geo.Nb * kept * sizeof(int32_t),
+                        cudaMemcpyDeviceToDevice, s);
+  if (e != cudaSuccess) return RF2_ERR_CUDA;
+  return finish_checked(flags, w.mask.status, s);
+}
+
+}  // extern "C"

@@ -1,0 +1,98 @@
+// Shared host/device definitions of the sm_100a block-sparse attention library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "rf2.h"
+
+namespace rf2 {
+
+// Derived geometry of one call (host-computed, passed to kernels by value).
+// Blocks are (wt, wh, ww) windows of the grid padded at the high end of each axis,
+// numbered row-major over (t/wt, h/wh, w/ww); tokens inside a window are row-major
+// over (t%wt, h%wh, w%ww) ("3D window permutation", RainFusion2.0 TL;DR).
+struct Geo {
+  int B, heads, T, H, W, D, wt, wh, ww;
+  int nbt, nbh, nbw;  // windows per axis
+  int Nb, blk;        // blocks, tokens per block
+  long long N, Npad;  // real tokens, padded tokens (per batch)
+};
+
+inline Geo make_geo(const rf2_geom& g) {
+  Geo o;
+  o.B = g.B; o.heads = g.heads; o.T = g.T; o.H = g.H; o.W = g.W; o.D = g.D;
+  o.wt = g.wt; o.wh = g.wh; o.ww = g.ww;
+  o.nbt = (g.T + g.wt - 1) / g.wt;
+  o.nbh = (g.H + g.wh - 1) / g.wh;
+  o.nbw = (g.W + g.ww - 1) / g.ww;
+  o.Nb = o.nbt * o.nbh * o.nbw;
+  o.blk = g.wt * g.wh * g.ww;
+  o.N = (long long)g.T * g.H * g.W;
+  o.Npad = (long long)o.Nb * o.blk;
+  return o;
+}
+
+// Raster token of permuted position p (within one batch), or -1 for a pad position.
+__host__ __device__ __forceinline__ long long pos_to_token(const Geo& g, long long p) {
+  int block = (int)(p / g.blk);
+  int off = (int)(p - (long long)block * g.blk);
+  int per_t = g.nbh * g.nbw;
+  int tb = block / per_t;
+  int rem = block - tb * per_t;
+  int hb = rem / g.nbw;
+  int wb = rem - hb * g.nbw;
+  int whw = g.wh * g.ww;
+  int dt = off / whw;
+  int r2 = off - dt * whw;
+  int dh = r2 / g.ww;
+  int dw = r2 - dh * g.ww;
+  int t = tb * g.wt + dt, h = hb * g.wh + dh, w = wb * g.ww + dw;
+  if (t >= g.T || h >= g.H || w >= g.W) return -1;
+  return ((long long)t * g.H + h) * g.W + w;
+}
+
+// Permuted position of raster token n (within one batch).
+__host__ __device__ __forceinline__ long long token_to_pos(const Geo& g, long long n) {
+  int w = (int)(n % g.W);
+  long long th = n / g.W;
+  int h = (int)(th % g.H);
+  int t = (int)(th / g.H);
+  int block = ((t / g.wt) * g.nbh + h / g.wh) * g.nbw + w / g.ww;
+  int off = ((t % g.wt) * g.wh + h % g.wh) * g.ww + w % g.ww;
+  return (long long)block * g.blk + off;
+}
+
+// Real tokens of block j and, per axis, how many of the window's rows are real.
+__host__ __device__ __forceinline__ void block_extent(const Geo& g, int j, int& nt, int& nh,
+                                                      int& nw) {
+  int per_t = g.nbh * g.nbw;
+  int tb = j / per_t;
+  int rem = j - tb * per_t;
+  int hb = rem / g.nbw;
+  int wb = rem - hb * g.nbw;
+  nt = min(g.wt, g.T - tb * g.wt);
+  nh = min(g.wh, g.H - hb * g.wh);
+  nw = min(g.ww, g.W - wb * g.ww);
+}
+
+// Device status word values (match rf2_status).
+constexpr int kStatusBadIndex = RF2_ERR_BAD_INDEX;
+constexpr int kStatusTimeout = RF2_ERR_TIMEOUT;
+
+// Launchers (defined in the kernel files, called by the C ABI layer).
+cudaError_t launch_permute(const void* x, void* xp, const Geo& g, cudaStream_t s);
+cudaError_t launch_unpermute(const void* xp, void* x, const Geo& g, cudaStream_t s);
+cudaError_t launch_pool(const void* qp, const void* kp, float* qbar, float* kbar, const Geo& g,
+                        cudaStream_t s);
+cudaError_t launch_scores(const float* qbar, const float* kbar, float* scores, const Geo& g,
+                          float scale, cudaStream_t s);
+cudaError_t launch_topk(const float* scores, int32_t* idx, int32_t* cnt, int kmax, int kept,
+                        int nsink, const Geo& g, cudaStream_t s);
+// Returns cudaErrorNotSupported when the shape has no kernel instance.
+cudaError_t launch_sparse_attn(const void* qp, const void* kp, const void* vp,
+                               const int32_t* idx, const int32_t* cnt, int kmax, const Geo& g,
+                               float scale, void* op, int32_t* status, cudaStream_t s);
+
+}  // namespace rf2

@@ -1,0 +1,148 @@
+/*
+ * rf2.h - C ABI of the B200 (sm_100a) block-sparse attention library (librf2.so).
+ *
+ * The library computes the online block-sparse attention of RainFusion2.0
+ * ("RainFusion2.0: Temporal-Spatial Awareness and Hardware-Efficient Block-wise Sparse
+ * Attention"): a 3D-window token permutation of a [T, H, W] latent token grid, block-mean
+ * representative tokens for Q and K, a pooled block-level score that selects, per
+ * (batch, head, query block), the key blocks to keep at a target sparsity, a first-frame
+ * sink that always keeps the key blocks of the first temporal window, attention over the
+ * kept blocks only, and the inverse permutation.  Passages that define each step are
+ * cited per entry point below (mlsanity index page, Abstract, "key technical insights"
+ * (1)-(3); sciencestack page, TL;DR and Figures 1-3).  The pages give no formulas; the
+ * readings used here are stated with each call.
+ *
+ * Conventions (every entry point):
+ *  - Tensors are device pointers to contiguous row-major arrays.  Q/K/V/O in model order
+ *    are [B, N, heads, D] bf16 with N = T*H*W tokens in raster (t, h, w) order.  Permuted
+ *    tensors are [B, Npad, heads, D] bf16, Npad = Nb*blk, tokens in window order.
+ *  - The caller owns every buffer.  No entry point allocates memory or synchronises
+ *    the stream, except that RF2_CHECKED makes a call wait for its own work on `stream`
+ *    and read the device status word back.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  All work
+ *    is asynchronous on it.
+ *  - Arguments are validated on the host before any launch; an invalid call returns an
+ *    error and launches nothing.  Device pointers must be 16-byte aligned.
+ *  - Supported: D in {64, 128}; blk = wt*wh*ww in {64, 128}; B, heads, T, H, W >= 1.
+ *  - Return value: RF2_OK or an rf2_status error code.  A CUDA launch error maps to
+ *    RF2_ERR_CUDA.
+ */
+#ifndef RF2_H
+#define RF2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Geometry of one attention call.  The grid is padded at the high end of each axis to
+ * window multiples: Tp = ceil(T/wt)*wt (same for H, W).  Blocks are windows numbered
+ * row-major over (t/wt, h/wh, w/ww); Nb = (Tp/wt)*(Hp/wh)*(Wp/ww), blk = wt*wh*ww. */
+typedef struct rf2_geom {
+    int B, heads, T, H, W, D, wt, wh, ww;
+} rf2_geom;
+
+enum rf2_status {
+    RF2_OK = 0,
+    RF2_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, kmax too small ...   */
+    RF2_ERR_UNSUPPORTED = 2,  /* D or block size outside the supported set              */
+    RF2_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned                       */
+    RF2_ERR_WORKSPACE = 4,    /* workspace missing or smaller than the size query says  */
+    RF2_ERR_BAD_INDEX = 5,    /* a block index outside [0, Nb) (detected on device)      */
+    RF2_ERR_TIMEOUT = 6,      /* a bounded device wait gave up (detected on device)      */
+    RF2_ERR_CUDA = 7          /* a CUDA runtime error                                   */
+};
+
+enum rf2_flags {
+    /* Sink outside the budget: kept = |S| + ceil((1-s)*(Nb-|S|) - 1e-6).  Default is the
+     * in-budget reading: kept = max(ceil((1-s)*Nb - 1e-6) clamped to [1,Nb], |S|). */
+    RF2_SINK_ADDITIVE = 1u,
+    /* Wait for the call's work on `stream` and return the device status word. */
+    RF2_CHECKED = 2u
+};
+
+/* rf2_permute - 3D window permutation (mlsanity index page, Abstract, insight (2)
+ * "spatiotemporal-aware token permutation"; sciencestack page, TL;DR "3D window
+ * permutation" and Figure 3).
+ *   x  : [B, N, heads, D] bf16, raster order (read).
+ *   xp : [B, Npad, heads, D] bf16 (written).  Token (t,h,w) goes to position
+ *        block*blk + ((t%wt)*wh + h%wh)*ww + w%ww, block = ((t/wt)*(Hp/wh) + h/wh)*(Wp/ww)
+ *        + w/ww.  Pad positions are written with zeros.
+ * Errors: RF2_ERR_INVALID_ARG, RF2_ERR_UNSUPPORTED, RF2_ERR_ALIGNMENT, RF2_ERR_CUDA. */
+int rf2_permute(const void* x, void* xp, const rf2_geom* g, void* stream);
+
+/* rf2_unpermute - inverse of rf2_permute; pad positions are dropped.
+ *   xp : [B, Npad, heads, D] bf16 (read).   x : [B, N, heads, D] bf16 (written). */
+int rf2_unpermute(const void* xp, void* x, const rf2_geom* g, void* stream);
+
+/* rf2_kept_count - number of key blocks every (b, head, query block) row keeps
+ * (sciencestack page, TL;DR: target sparsity; mlsanity index page, insight (3): the
+ * first-frame sink).  The sink S is the Hp/wh * Wp/ww blocks of temporal window 0 when
+ * `sink` is non-zero.  Returns the count (>= 1) or -RF2_ERR_* on a bad argument.
+ * This is the minimum `kmax` of rf2_predict_mask. */
+int rf2_kept_count(const rf2_geom* g, double sparsity, int sink, unsigned flags);
+
+/* rf2_workspace_size - bytes of device workspace that rf2_predict_mask (attention = 0)
+ * or rf2_attention (attention = 1) needs for this geometry, sparsity and flags.  The
+ * workspace holds the pooled block means, pooled scores, the kept lists (attention) and
+ * the permuted Q/K/V/O copies (attention), plus a status word.  Returns 0 on a bad
+ * argument. */
+size_t rf2_workspace_size(const rf2_geom* g, double sparsity, int sink, unsigned flags,
+                          int attention);
+
+/* rf2_predict_mask - online mask prediction on permuted Q and K (mlsanity index page,
+ * Abstract, insight (1) "block-wise mean values as representative tokens for sparse mask
+ * prediction" and insight (3) "first-frame sink").
+ *   qp, kp : [B, Npad, heads, D] bf16, window order (read).  Pad positions are ignored.
+ *   Steps: qbar_i, kbar_j = fp32 mean over the real tokens of each block, per head;
+ *   s_ij = qbar_i . kbar_j / sqrt(D) (fp32); each row keeps the sink blocks plus the
+ *   highest-scoring other blocks (ties to the lower id) up to rf2_kept_count.
+ *   idx : [B, heads, Nb, kmax] int32 (written): ascending kept block ids, then -1.
+ *   cnt : [B, heads, Nb] int32 (written): the kept count of each row.
+ *   kmax >= rf2_kept_count(...) else RF2_ERR_INVALID_ARG.
+ *   ws, ws_bytes : device scratch of at least rf2_workspace_size(..., 0) bytes.
+ * Errors: RF2_ERR_INVALID_ARG, RF2_ERR_UNSUPPORTED, RF2_ERR_ALIGNMENT, RF2_ERR_WORKSPACE,
+ *         RF2_ERR_CUDA. */
+int rf2_predict_mask(const void* qp, const void* kp, const rf2_geom* g, double sparsity,
+                     int sink, unsigned flags, int32_t* idx, int32_t* cnt, int kmax,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* rf2_sparse_attn - block-sparse attention over the kept blocks (mlsanity index page,
+ * title "block-wise sparse attention"; Abstract: skipping the computation of
+ * insignificant tokens).  For each (b, head, query block i):
+ *   O_i = softmax(Q_i K_S^T * scale + M) V_S over the tokens of the kept blocks
+ *   S = idx[b, head, i, 0..cnt-1]; M = -inf on pad keys, 0 elsewhere.
+ *   qp, kp, vp : [B, Npad, heads, D] bf16 (read).   op : [B, Npad, heads, D] bf16
+ *   (written; pad query rows are written too, with values of no meaning).
+ *   scale : softmax scale; 0 means 1/sqrt(D).  Softmax statistics and the accumulator
+ *   are fp32; P is rounded to bf16 for the P.V product.
+ *   status : optional device int32 (may be NULL); when given it must be zero on entry
+ *   and receives RF2_ERR_BAD_INDEX / RF2_ERR_TIMEOUT if the kernel detects one
+ *   (out-of-range ids are skipped, never dereferenced).  With RF2_CHECKED and a status
+ *   word the call waits for the stream and returns that code.
+ * Errors: RF2_ERR_INVALID_ARG, RF2_ERR_UNSUPPORTED, RF2_ERR_ALIGNMENT, RF2_ERR_CUDA,
+ *         and (checked mode) RF2_ERR_BAD_INDEX, RF2_ERR_TIMEOUT. */
+int rf2_sparse_attn(const void* qp, const void* kp, const void* vp, const int32_t* idx,
+                    const int32_t* cnt, int kmax, const rf2_geom* g, float scale, void* op,
+                    int32_t* status, unsigned flags, void* stream);
+
+/* rf2_attention - the whole path (sciencestack page, Figure 1 "Workflow of
+ * RainFusion2.0"): permute Q/K/V -> predict mask -> block-sparse attention -> unpermute.
+ *   q, k, v : [B, N, heads, D] bf16 (read).   o : [B, N, heads, D] bf16 (written).
+ *   idx_out : optional [B, heads, Nb, kept] int32 copy of the kept lists (may be NULL).
+ *   ws, ws_bytes : device scratch of at least rf2_workspace_size(..., 1) bytes.
+ * Errors: as rf2_predict_mask and rf2_sparse_attn. */
+int rf2_attention(const void* q, const void* k, const void* v, const rf2_geom* g,
+                  double sparsity, int sink, float scale, void* o, int32_t* idx_out,
+                  void* ws, size_t ws_bytes, unsigned flags, void* stream);
+
+/* rf2_status_string - static, human-readable text of a status code. */
+const char* rf2_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RF2_H */

@@ -39,6 +39,7 @@ so the method's outputs beyond these pins are "parity unpinned by the pages".
 """
 from __future__ import annotations
 
+import functools
 import math
 from dataclasses import dataclass
 from typing import List, Optional, Sequence, Tuple
@@ -120,6 +121,7 @@ def window_positions(g: Geom) -> np.ndarray:
     return block * g.blk + offset
 
 
+@functools.lru_cache(maxsize=32)
 def position_to_token(g: Geom) -> np.ndarray:
     """Inverse map, built independently of window_positions: for every permuted position
     p in [0, Npad), the raster token index (t*H + h)*W + w, or -1 for a pad position."""
@@ -133,6 +135,7 @@ def position_to_token(g: Geom) -> np.ndarray:
         t, h, w = tb * g.wt + dt, hb * g.wh + dh, wb * g.ww + dw
         if t < g.T and h < g.H and w < g.W:
             out[p] = (t * g.H + h) * g.W + w
+    out.setflags(write=False)
     return out
 
 

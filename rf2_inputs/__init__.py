@@ -17,8 +17,9 @@ Generator (one tensor X of shape [B, N, heads, D], tokens in raster (t, h, w) or
 
 with (ft, fh, fw, phi) drawn per (head, c, j): ft ~ U[0.5, 2], fh, fw ~ U[0.5, 4],
 phi ~ U[0, 2*pi).  Var F is about 1, so block means carry real spatial structure.
-Parameters come from numpy's PCG64 with seed ``1000 * cfg + {0, 1, 2}`` for Q/K/V;
-the field is evaluated in float32 and the sum rounded to bf16 (round to nearest even).
+Parameters come from numpy's PCG64 with seed ``1000 * cfg + {0, 1, 2}`` for Q/K/V and
+the noise from torch's CPU generator with the same seed; angles and their sin/cos in
+float64, the field and the noise in float32, the sum rounded to bf16 (nearest even).
 """
 from __future__ import annotations
 
@@ -33,6 +34,7 @@ __all__ = [
     "workload",
     "gen_tensor",
     "gen_qkv",
+    "gen_tensor_torch",
     "bf16_bits_to_f64",
     "f32_to_bf16_bits",
 ]
@@ -102,26 +104,43 @@ def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
 
 def gen_tensor(B: int, T: int, H: int, W: int, heads: int, D: int, seed: int,
                field_amp: float = 0.5, noise: float = 1.0, n_sin: int = 4) -> np.ndarray:
-    """Return raw bf16 bits (uint16) of shape [B, T*H*W, heads, D], raster token order."""
+    """Return raw bf16 bits (uint16) of shape [B, T*H*W, heads, D], raster token order.
+
+    Each sinusoid is evaluated through the angle-addition identity,
+    sin(a_t + b_h + c_w) = sin(a_t + b_h) cos(c_w) + cos(a_t + b_h) sin(c_w),
+    so that only [H, heads*D] and [W, heads*D] tables need sin/cos (float64) and the
+    [H, W] field of each frame is one small batched product (float32).  The noise is
+    drawn by torch's CPU generator seeded with the same seed; CPU tensors only."""
+    import torch
+
     rng = np.random.Generator(np.random.PCG64(seed))
-    ft = rng.uniform(0.5, 2.0, size=(B, heads, D, n_sin)).astype(np.float32)
-    fh = rng.uniform(0.5, 4.0, size=(B, heads, D, n_sin)).astype(np.float32)
-    fw = rng.uniform(0.5, 4.0, size=(B, heads, D, n_sin)).astype(np.float32)
-    ph = rng.uniform(0.0, 2.0 * np.pi, size=(B, heads, D, n_sin)).astype(np.float32)
-    amp = np.float32(field_amp / np.sqrt(2.0))
-    two_pi = np.float32(2.0 * np.pi)
-    hh = (np.arange(H, dtype=np.float32) / np.float32(H))[:, None, None, None, None]
-    ww = (np.arange(W, dtype=np.float32) / np.float32(W))[None, :, None, None, None]
-    out = np.empty((B, T, H, W, heads, D), dtype=np.uint16)
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(int(seed))
+    C = heads * D
+    ft = rng.uniform(0.5, 2.0, size=(B, C, n_sin))
+    fh = rng.uniform(0.5, 4.0, size=(B, C, n_sin))
+    fw = rng.uniform(0.5, 4.0, size=(B, C, n_sin))
+    ph = rng.uniform(0.0, 2.0 * np.pi, size=(B, C, n_sin))
+    amp = field_amp / np.sqrt(2.0)
+    two_pi = 2.0 * np.pi
+    hh = (np.arange(H) / H)[:, None, None]
+    ww = (np.arange(W) / W)[:, None, None]
+    out = torch.empty((B, T, H, W, C), dtype=torch.bfloat16)
     for b in range(B):
-        # phase over (h, w, head, c, j), without the t term
-        base = two_pi * (fh[b][None, None] * hh + fw[b][None, None] * ww) + ph[b][None, None]
+        cw = two_pi * fw[b][None] * ww                      # [W, C, n]
+        qw = np.concatenate([np.cos(cw), np.sin(cw)], axis=-1)
+        qw = torch.from_numpy(np.ascontiguousarray(qw.transpose(1, 2, 0), dtype=np.float32))  # [C,2n,W]
         for t in range(T):
-            ang = base + two_pi * ft[b] * np.float32(t / T)
-            field = amp * np.sin(ang, dtype=np.float32).sum(axis=-1, dtype=np.float32)
-            eps = rng.standard_normal(size=(H, W, heads, D), dtype=np.float32)
-            out[b, t] = f32_to_bf16_bits(field + np.float32(noise) * eps)
-    return out.reshape(B, T * H * W, heads, D)
+            ah = two_pi * (ft[b][None] * (t / T) + fh[b][None] * hh) + ph[b][None]  # [H, C, n]
+            pa = np.concatenate([np.sin(ah), np.cos(ah)], axis=-1) * amp
+            pa = torch.from_numpy(np.ascontiguousarray(pa.transpose(1, 0, 2), dtype=np.float32))  # [C,H,2n]
+            field = torch.bmm(pa, qw).permute(1, 2, 0)                                           # [H,W,C]
+            x = torch.randn((H, W, C), generator=gen, dtype=torch.float32)
+            if noise != 1.0:
+                x.mul_(noise)
+            x.add_(field)
+            out[b, t] = x.to(torch.bfloat16)
+    return out.view(torch.int16).numpy().view(np.uint16).reshape(B, T * H * W, heads, D)
 
 
 def gen_qkv(wl: Workload, seed_base: Optional[int] = None,
@@ -130,3 +149,38 @@ def gen_qkv(wl: Workload, seed_base: Optional[int] = None,
     s0 = 1000 * wl.cfg if seed_base is None else seed_base
     B = wl.B if batch is None else batch
     return [gen_tensor(B, wl.T, wl.H, wl.W, wl.heads, wl.D, s0 + i) for i in range(3)]
+
+
+def gen_tensor_torch(B: int, T: int, H: int, W: int, heads: int, D: int, seed: int,
+                     device, field_amp: float = 0.5, n_sin: int = 4):
+    """The same recipe as gen_tensor, evaluated with torch on `device` (used to build
+    large benchmark inputs quickly).  The field parameters are identical to gen_tensor's;
+    the noise comes from the device's generator, so the bits differ from gen_tensor's.
+    Returns a bf16 tensor [B, T*H*W, heads, D] on `device`."""
+    import torch
+
+    rng = np.random.Generator(np.random.PCG64(seed))
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    C = heads * D
+    ft = rng.uniform(0.5, 2.0, size=(B, C, n_sin))
+    fh = rng.uniform(0.5, 4.0, size=(B, C, n_sin))
+    fw = rng.uniform(0.5, 4.0, size=(B, C, n_sin))
+    ph = rng.uniform(0.0, 2.0 * np.pi, size=(B, C, n_sin))
+    amp = field_amp / np.sqrt(2.0)
+    two_pi = 2.0 * np.pi
+    hh = (np.arange(H) / H)[:, None, None]
+    ww = (np.arange(W) / W)[:, None, None]
+    out = torch.empty((B, T, H, W, C), dtype=torch.bfloat16, device=device)
+    for b in range(B):
+        cw = two_pi * fw[b][None] * ww
+        qw = np.concatenate([np.cos(cw), np.sin(cw)], axis=-1)
+        qw = torch.from_numpy(np.ascontiguousarray(qw.transpose(1, 2, 0), dtype=np.float32)).to(device)
+        for t in range(T):
+            ah = two_pi * (ft[b][None] * (t / T) + fh[b][None] * hh) + ph[b][None]
+            pa = np.concatenate([np.sin(ah), np.cos(ah)], axis=-1) * amp
+            pa = torch.from_numpy(np.ascontiguousarray(pa.transpose(1, 0, 2), dtype=np.float32)).to(device)
+            x = torch.randn((H, W, C), generator=gen, dtype=torch.float32, device=device)
+            x.add_(torch.bmm(pa, qw).permute(1, 2, 0))
+            out[b, t] = x.to(torch.bfloat16)
+    return out.view(B, T * H * W, heads, D)

@@ -1,0 +1,130 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every symbol
+include/rf2.h declares, and rejects bad arguments before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle as O
+import image_diffusion_dits_b200 as rf2
+from image_diffusion_dits_b200 import _lib
+from rf2_inputs import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(rf2_[a-z_0-9]+)\s*\(", src))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    declared = _declared()
+    assert declared, "no declarations found"
+    assert declared == set(_lib.EXPORTS)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def _g(**kw):
+    base = dict(B=1, heads=2, T=4, H=16, W=16, D=64, wt=1, wh=8, ww=8)
+    base.update(kw)
+    return rf2.Geometry(**base)
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_kept_count_matches_oracle(name):
+    wl = WORKLOADS[name]
+    g = rf2.Geometry(**wl.geom())
+    og = O.geom(**wl.geom())
+    for s in wl.sparsities:
+        for additive in (False, True):
+            assert rf2.kept_count(g, s, wl.sink, additive) == O.kept_count(og, s, wl.sink, additive)
+            assert rf2.kept_count(g, s, not wl.sink, additive) == O.kept_count(og, s, not wl.sink, additive)
+
+
+def test_kept_count_sweep_matches_oracle():
+    og = O.geom(B=1, heads=1, T=31, H=45, W=80, D=128, wt=2, wh=8, ww=8)
+    g = rf2.Geometry(**og.__dict__)
+    for i in range(0, 101):
+        s = i / 100
+        for sink in (False, True):
+            for additive in (False, True):
+                assert rf2.kept_count(g, s, sink, additive) == O.kept_count(og, s, sink, additive), (s, sink, additive)
+
+
+def test_workspace_size_covers_buffers():
+    wl = WORKLOADS["wan720p"]
+    g = rf2.Geometry(**wl.geom())
+    ws_attn = rf2.workspace_size(g, 0.8, True)
+    ws_mask = rf2.workspace_size(g, 0.8, True, attention=False)
+    t = g.B * g.Npad * g.heads * g.D * 2
+    assert ws_mask >= 2 * g.B * g.heads * g.Nb * g.D * 4 + g.B * g.heads * g.Nb * g.Nb * 4
+    assert ws_attn >= ws_mask + 4 * t + g.B * g.heads * g.Nb * 132 * 4
+
+
+def _call_status(fn, *args):
+    return fn(*args)
+
+
+def test_invalid_arguments_are_rejected_without_launch():
+    lib = _lib.load()
+    good = _g().c()
+    p = 1 << 20  # a 16-byte-aligned fake address; never dereferenced (rejected first)
+    # null pointers
+    assert lib.rf2_permute(None, p, ctypes.byref(good), None) == _lib.RF2_ERR_INVALID_ARG
+    assert lib.rf2_unpermute(p, None, ctypes.byref(good), None) == _lib.RF2_ERR_INVALID_ARG
+    # misaligned pointers
+    assert lib.rf2_permute(p + 2, p, ctypes.byref(good), None) == _lib.RF2_ERR_ALIGNMENT
+    # unsupported head_dim / block size
+    bad_d = _g(D=96).c()
+    assert lib.rf2_permute(p, p, ctypes.byref(bad_d), None) == _lib.RF2_ERR_UNSUPPORTED
+    bad_blk = _g(wh=4).c()
+    assert lib.rf2_permute(p, p, ctypes.byref(bad_blk), None) == _lib.RF2_ERR_UNSUPPORTED
+    # non-positive sizes and null geometry
+    zero = _g(T=0).c()
+    assert lib.rf2_permute(p, p, ctypes.byref(zero), None) == _lib.RF2_ERR_INVALID_ARG
+    assert lib.rf2_permute(p, p, None, None) == _lib.RF2_ERR_INVALID_ARG
+    # kmax below the kept count
+    k = lib.rf2_kept_count(ctypes.byref(good), 0.8, 1, 0)
+    assert k == 4
+    assert lib.rf2_predict_mask(p, p, ctypes.byref(good), 0.8, 1, 0, p, p, k - 1, p, 1 << 30, None) == \
+        _lib.RF2_ERR_INVALID_ARG
+    # sparsity outside [0, 1]
+    assert lib.rf2_kept_count(ctypes.byref(good), 1.5, 1, 0) == -_lib.RF2_ERR_INVALID_ARG
+    assert lib.rf2_workspace_size(ctypes.byref(good), -0.1, 1, 0, 1) == 0
+    # workspace missing or too small
+    assert lib.rf2_predict_mask(p, p, ctypes.byref(good), 0.8, 1, 0, p, p, k, None, 0, None) == \
+        _lib.RF2_ERR_WORKSPACE
+    assert lib.rf2_predict_mask(p, p, ctypes.byref(good), 0.8, 1, 0, p, p, k, p, 16, None) == \
+        _lib.RF2_ERR_WORKSPACE
+    assert lib.rf2_attention(p, p, p, ctypes.byref(good), 0.8, 1, 0.0, p, None, p, 16, 0, None) == \
+        _lib.RF2_ERR_WORKSPACE
+    # non-finite scale
+    assert lib.rf2_sparse_attn(p, p, p, p, p, k, ctypes.byref(good), float("nan"), p, None, 0, None) == \
+        _lib.RF2_ERR_INVALID_ARG
+    # too many blocks for the kept-list capacity
+    big = _g(T=64, H=64, W=64).c()  # 4096 blocks
+    assert lib.rf2_permute(p, p, ctypes.byref(big), None) == _lib.RF2_ERR_UNSUPPORTED
+
+
+def test_status_strings():
+    lib = _lib.load()
+    for code in range(8):
+        assert lib.rf2_status_string(code)
+    assert b"unknown" in lib.rf2_status_string(99)
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    g = _g()
+    x = torch.zeros((1, g.N, g.heads, g.D), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        rf2.permute(x, g)

@@ -1,0 +1,259 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle on the same
+seeded bf16 inputs.  Permutations and kept lists are compared bit-exactly (kept lists
+outside the near-cut window); attention outputs within max-abs 2e-2 and relative-L2 1e-2."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import image_diffusion_dits_b200 as rf2
+from rf2_inputs import WORKLOADS, bf16_bits_to_f64, gen_qkv, gen_tensor
+
+from _util import assert_close, compare_lists, to_bits, to_dev, to_f64
+
+pytestmark = pytest.mark.gpu
+
+SMALL = ["tiny", "video480p", "imgedit1024"]
+LARGE = ["wan720p", "longvideo"]
+
+_cache = {}
+
+
+def _inputs(name):
+    if name not in _cache:
+        _cache.clear()
+        _cache[name] = gen_qkv(WORKLOADS[name])
+    return _cache[name]
+
+
+def _geoms(name):
+    wl = WORKLOADS[name]
+    return wl, rf2.Geometry(**wl.geom()), O.geom(**wl.geom())
+
+
+# Ragged shapes: padding on every axis, both block sizes, both head dims, batch > 1.
+RAGGED = [
+    dict(B=2, heads=3, T=3, H=7, W=10, D=64, wt=1, wh=8, ww=8),
+    dict(B=1, heads=2, T=5, H=9, W=17, D=128, wt=2, wh=8, ww=8),
+    dict(B=2, heads=1, T=3, H=13, W=9, D=128, wt=1, wh=8, ww=8),
+    dict(B=1, heads=2, T=4, H=11, W=21, D=64, wt=2, wh=4, ww=16),
+    dict(B=1, heads=1, T=1, H=8, W=8, D=64, wt=1, wh=8, ww=8),      # one block
+    dict(B=1, heads=2, T=2, H=16, W=23, D=128, wt=1, wh=8, ww=16),
+]
+
+
+def _rand_bits(g, seed):
+    return [gen_tensor(g.B, g.T, g.H, g.W, g.heads, g.D, seed + i) for i in range(3)]
+
+
+# ----------------------------------------------------------------------------- permutation
+
+@pytest.mark.parametrize("shape", RAGGED)
+def test_permute_unpermute_ragged_bit_exact(shape):
+    g, og = rf2.Geometry(**shape), O.geom(**shape)
+    x = _rand_bits(g, 101)[0]
+    xd = to_dev(x)
+    xp = rf2.permute(xd, g)
+    np.testing.assert_array_equal(to_bits(xp), O.permute(x, og))
+    back = rf2.unpermute(xp, g)
+    np.testing.assert_array_equal(to_bits(back), x)
+
+
+@pytest.mark.parametrize("name", SMALL + LARGE)
+def test_permute_unpermute_workloads_bit_exact(name):
+    wl, g, og = _geoms(name)
+    q, _, _ = _inputs(name)
+    xp = rf2.permute(to_dev(q), g)
+    np.testing.assert_array_equal(to_bits(xp), O.permute(q, og))
+    np.testing.assert_array_equal(to_bits(rf2.unpermute(xp, g)), q)
+
+
+def test_permute_overwrites_pad_rows_with_zero():
+    shape = RAGGED[0]
+    g, og = rf2.Geometry(**shape), O.geom(**shape)
+    x = to_dev(_rand_bits(g, 7)[0])
+    out = torch.full((g.B, g.Npad, g.heads, g.D), 3.0, dtype=torch.bfloat16, device="cuda")
+    rf2.permute(x, g, out=out)
+    pad = ~O.position_valid(og)
+    assert torch.all(out[:, torch.from_numpy(pad).cuda()] == 0)
+
+
+# ----------------------------------------------------------------------------- mask prediction
+
+def _mask_case(name_or_shape, sparsity, sink, additive, seed=None):
+    if isinstance(name_or_shape, str):
+        wl, g, og = _geoms(name_or_shape)
+        q, k, _ = _inputs(name_or_shape)
+    else:
+        g, og = rf2.Geometry(**name_or_shape), O.geom(**name_or_shape)
+        q, k, _ = _rand_bits(g, seed)
+    qp, kp = O.permute(q, og), O.permute(k, og)
+    sel = O.predict_mask(bf16_bits_to_f64(qp), bf16_bits_to_f64(kp), og, sparsity, sink, additive)
+    idx, cnt = rf2.predict_mask(to_dev(qp), to_dev(kp), g, sparsity, sink, additive,
+                                kmax=sel.kept + 3, checked=True)
+    return compare_lists(idx.cpu().numpy(), cnt.cpu().numpy(), sel)
+
+
+@pytest.mark.parametrize("shape", RAGGED)
+@pytest.mark.parametrize("additive", [False, True])
+def test_predict_mask_ragged(shape, additive):
+    for s, sink in ((0.8, True), (0.5, False), (0.0, True), (1.0, True)):
+        _mask_case(shape, s, sink, additive, seed=300)
+
+
+@pytest.mark.parametrize("name", SMALL + LARGE)
+@pytest.mark.parametrize("additive", [False, True])
+def test_predict_mask_workloads(name, additive):
+    wl = WORKLOADS[name]
+    for s in wl.sparsities:
+        stats = _mask_case(name, s, wl.sink, additive)
+        print(name, s, "additive" if additive else "in-budget", stats)
+
+
+# ----------------------------------------------------------------------------- sparse attention
+
+def _attn_case(g, og, q, k, v, sparsity, sink, heads=None, rows=None, scale=0.0):
+    """Oracle kept lists feed both sides; compare all heads (or sampled (head, q-block))."""
+    qp, kp, vp = (O.permute(a, og) for a in (q, k, v))
+    qf, kf, vf = (bf16_bits_to_f64(a) for a in (qp, kp, vp))
+    sel = O.predict_mask(qf, kf, og, sparsity, sink)
+    idx = torch.from_numpy(sel.idx).cuda()
+    cnt = torch.full(sel.idx.shape[:3], sel.kept, dtype=torch.int32, device="cuda")
+    op = rf2.sparse_attn(to_dev(qp), to_dev(kp), to_dev(vp), idx, cnt, g, scale=scale, checked=True)
+    got = to_f64(op)
+    sc = O.default_scale(og.D, scale)
+    valid = O.position_valid(og)
+    if rows is None:
+        hs = range(og.heads) if heads is None else heads
+        rows = [(b, h, i) for b in range(og.B) for h in hs for i in range(og.Nb)]
+    ref_rows, got_rows = [], []
+    for (b, h, i) in rows:
+        ref = O.attention_block(qf, kf, vf, og, b, h, i, sel.idx[b, h, i], sc)
+        keep = valid[i * og.blk:(i + 1) * og.blk]
+        ref_rows.append(ref[keep])
+        got_rows.append(got[b, i * og.blk:(i + 1) * og.blk, h][keep])
+    return assert_close(np.concatenate(got_rows), np.concatenate(ref_rows), "sparse_attn")
+
+
+@pytest.mark.parametrize("shape", RAGGED)
+def test_sparse_attn_ragged(shape):
+    g, og = rf2.Geometry(**shape), O.geom(**shape)
+    q, k, v = (bf16_bits_to_f64(a) for a in _rand_bits(g, 500))
+    bits = _rand_bits(g, 500)
+    for s, sink in ((0.5, True), (0.0, False)):
+        _attn_case(g, og, *bits, s, sink)
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_sparse_attn_small_workloads_all_rows(name):
+    wl, g, og = _geoms(name)
+    q, k, v = _inputs(name)
+    stats = _attn_case(g, og, q, k, v, wl.sparsity, wl.sink)
+    print(name, stats)
+
+
+@pytest.mark.parametrize("name", LARGE)
+def test_sparse_attn_large_workloads_sampled_rows(name):
+    wl, g, og = _geoms(name)
+    q, k, v = _inputs(name)
+    rng = np.random.default_rng(17)
+    rows = {(0, int(rng.integers(og.heads)), int(rng.integers(og.Nb))) for _ in range(20)}
+    rows |= {(0, 0, 0), (0, og.heads - 1, og.Nb - 1), (0, 1, og.Nb - og.nbw)}  # first, last, partial
+    stats = _attn_case(g, og, q, k, v, wl.sparsity, wl.sink, rows=sorted(rows))
+    print(name, stats)
+
+
+def test_sparse_attn_zero_sparsity_is_dense_attention():
+    shape = dict(B=1, heads=2, T=3, H=9, W=10, D=64, wt=1, wh=8, ww=8)
+    g, og = rf2.Geometry(**shape), O.geom(**shape)
+    q, k, v = _rand_bits(g, 900)
+    out, idx = rf2.attention(to_dev(q), to_dev(k), to_dev(v), g, 0.0, True, return_idx=True)
+    ref = O.dense_attention(*(bf16_bits_to_f64(a) for a in (q, k, v)), 1 / np.sqrt(g.D))
+    assert_close(to_f64(out), ref, "dense")
+    assert np.all(idx.cpu().numpy() == np.arange(og.Nb))
+
+
+def test_sparse_attn_custom_scale():
+    shape = RAGGED[1]
+    g, og = rf2.Geometry(**shape), O.geom(**shape)
+    _attn_case(g, og, *_rand_bits(g, 910), 0.5, True, scale=0.05)
+
+
+def test_sparse_attn_bad_index_is_skipped_and_reported():
+    shape = dict(B=1, heads=1, T=2, H=16, W=16, D=64, wt=1, wh=8, ww=8)
+    g, og = rf2.Geometry(**shape), O.geom(**shape)
+    q, k, v = _rand_bits(g, 920)
+    qp, kp, vp = (to_dev(O.permute(a, og)) for a in (q, k, v))
+    idx = torch.tensor([[[[0, 3, 99], [1, -5, 2]] + [[0, 1, 2]] * (og.Nb - 2)]], dtype=torch.int32,
+                       device="cuda")
+    cnt = torch.full((1, 1, og.Nb), 3, dtype=torch.int32, device="cuda")
+    with pytest.raises(rf2.Rf2Error) as ei:
+        rf2.sparse_attn(qp, kp, vp, idx, cnt, g, checked=True)
+    assert ei.value.code == 5
+    # the valid ids of the bad rows are still used
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    op = rf2.sparse_attn(qp, kp, vp, idx, cnt, g, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 5
+    qf, kf, vf = (bf16_bits_to_f64(O.permute(a, og)) for a in (q, k, v))
+    ref0 = O.attention_block(qf, kf, vf, og, 0, 0, 0, [0, 3], 1 / 8)
+    ref1 = O.attention_block(qf, kf, vf, og, 0, 0, 1, [1, 2], 1 / 8)
+    got = to_f64(op)
+    assert_close(got[0, :64, 0], ref0, "row0")
+    assert_close(got[0, 64:128, 0], ref1, "row1")
+
+
+def test_sparse_attn_empty_row_writes_zeros_and_respects_cnt():
+    shape = dict(B=1, heads=1, T=2, H=16, W=16, D=128, wt=2, wh=8, ww=8)
+    g, og = rf2.Geometry(**shape), O.geom(**shape)
+    q, k, v = _rand_bits(g, 930)
+    qp, kp, vp = (to_dev(O.permute(a, og)) for a in (q, k, v))
+    idx = torch.tensor([[[[0, 1, 2, 3]] * og.Nb]], dtype=torch.int32, device="cuda")
+    cnt = torch.tensor([[[0, 2, 4, 1]]], dtype=torch.int32, device="cuda")
+    op = rf2.sparse_attn(qp, kp, vp, idx, cnt, g, checked=True)
+    got = to_f64(op)
+    assert np.all(got[0, :128] == 0)
+    qf, kf, vf = (bf16_bits_to_f64(O.permute(a, og)) for a in (q, k, v))
+    for i, lst in ((1, [0, 1]), (2, [0, 1, 2, 3]), (3, [0])):
+        ref = O.attention_block(qf, kf, vf, og, 0, 0, i, lst, 1 / np.sqrt(128))
+        assert_close(got[0, i * 128:(i + 1) * 128, 0], ref, f"row{i}")
+
+
+# ----------------------------------------------------------------------------- fused path
+
+@pytest.mark.parametrize("name", SMALL + ["wan720p"])
+def test_attention_end_to_end(name):
+    wl, g, og = _geoms(name)
+    q, k, v = _inputs(name)
+    out, idx = rf2.attention(to_dev(q), to_dev(k), to_dev(v), g, wl.sparsity, wl.sink,
+                             return_idx=True, checked=True)
+    qf, kf, vf = (bf16_bits_to_f64(O.permute(a, og)) for a in (q, k, v))
+    sel = O.predict_mask(qf, kf, og, wl.sparsity, wl.sink)
+    gidx = idx.cpu().numpy()
+    stats = compare_lists(gidx, np.full(gidx.shape[:3], sel.kept), sel)
+    got = to_f64(out)
+    pos = O.window_positions(og).reshape(-1)
+    rng = np.random.default_rng(5)
+    heads = range(og.heads) if og.heads * og.Nb <= 2000 else rng.choice(og.heads, 2, replace=False)
+    blocks = range(og.Nb) if og.heads * og.Nb <= 2000 else rng.choice(og.Nb, 12, replace=False)
+    tok = O.position_to_token(og)
+    got_rows, ref_rows = [], []
+    for h in heads:
+        for i in blocks:
+            if not np.array_equal(gidx[0, h, i], sel.idx[0, h, i]):
+                continue  # near-cut difference in the kept set: not comparable
+            ref = O.attention_block(qf, kf, vf, og, 0, h, i, sel.idx[0, h, i], 1 / np.sqrt(og.D))
+            t = tok[i * og.blk:(i + 1) * og.blk]
+            keep = t >= 0
+            ref_rows.append(ref[keep])
+            got_rows.append(got[0, t[keep], h])
+    print(name, stats, assert_close(np.concatenate(got_rows), np.concatenate(ref_rows), name))
+    del pos
+
+
+def test_attention_is_deterministic():
+    wl, g, og = _geoms("video480p")
+    q, k, v = (to_dev(a) for a in _inputs("video480p"))
+    a = rf2.attention(q, k, v, g, 0.8, True)
+    b = rf2.attention(q, k, v, g, 0.8, True)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
