@@ -18,6 +18,7 @@ RF2_ERR_CUDA = 7
 
 RF2_SINK_ADDITIVE = 1
 RF2_CHECKED = 2
+RF2_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 # Every symbol include/rf2.h declares.
 EXPORTS = (
@@ -26,6 +27,7 @@ EXPORTS = (
     "rf2_kept_count",
     "rf2_workspace_size",
     "rf2_predict_mask",
+    "rf2_predict_mask_noalloc",
     "rf2_sparse_attn",
     "rf2_attention",
     "rf2_status_string",
@@ -48,6 +50,8 @@ _SIGS = {
                                              ctypes.c_int]),
     "rf2_predict_mask": (ctypes.c_int, [_vp, _vp, _gp, ctypes.c_double, ctypes.c_int, ctypes.c_uint,
                                         _i32p, _i32p, ctypes.c_int, _vp, ctypes.c_size_t, _vp]),
+    "rf2_predict_mask_noalloc": (ctypes.c_int, [_vp, _vp, _gp, ctypes.c_double, ctypes.c_int,
+                                                ctypes.c_uint, _i32p, _i32p, ctypes.c_int, _vp]),
     "rf2_sparse_attn": (ctypes.c_int, [_vp, _vp, _vp, _i32p, _i32p, ctypes.c_int, _gp, ctypes.c_float,
                                        _vp, _i32p, ctypes.c_uint, _vp]),
     "rf2_attention": (ctypes.c_int, [_vp, _vp, _vp, _gp, ctypes.c_double, ctypes.c_int, ctypes.c_float,

@@ -1,0 +1,90 @@
+// rf2_predict_mask_noalloc: the mask prediction of rf2_predict_mask for callers that
+// cannot allocate device memory.
+//
+// Some callers cannot call cudaMalloc at all: code that runs inside a framework that
+// owns every device allocation (a caching allocator, an inference runtime with a fixed
+// memory plan), or a plug-in loaded into a process that forbids allocation after its
+// start-up phase.  They can still pass their inputs and outputs, but not the scratch
+// that rf2_predict_mask takes as `ws`.  This entry point keeps that scratch in a
+// file-scope device array of fixed size instead, so it allocates nothing per call.
+//
+// The array (kScratchBytes) exists on every GPU that loads this library, from module
+// load until the process exits.  Every call on a device shares it and it keeps the last
+// call's contents; nothing in it has to start at zero, because each call writes every
+// byte it reads (block means, then pooled scores) before reading it.  Calls whose work
+// overlaps on the GPU (on different streams, or different host threads, of the same
+// device) race on the array and must be serialised by the caller.
+#include <math.h>
+
+#include <mutex>
+
+#include "rf2_common.cuh"
+
+namespace {
+
+constexpr size_t kScratchBytes = RF2_NOALLOC_SCRATCH_BYTES;
+constexpr size_t kAlign = 256;
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
+
+// Device address of g_scratch per device.  In host code the name g_scratch is only a
+// host-side stand-in; a kernel given it would fault, or read host memory where the GPU
+// can reach it.  The address is looked up once per device, with that device current.
+void* g_scratch_addr[kMaxDevices] = {nullptr};
+std::mutex g_scratch_mutex;
+
+int scratch_for_current_device(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RF2_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return RF2_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return RF2_OK;
+}
+
+size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" int rf2_predict_mask_noalloc(const void* qp, const void* kp, const rf2_geom* g,
+                                        double sparsity, int sink, unsigned flags, int32_t* idx,
+                                        int32_t* cnt, int kmax, void* stream) {
+  // Same argument rules as rf2_predict_mask; its size query gives the scratch needed.
+  const int kept = rf2_kept_count(g, sparsity, sink, flags);  // checks g and sparsity
+  if (kept < 0) return -kept;
+  const size_t need = rf2_workspace_size(g, sparsity, sink, flags, 0);
+  if (need == 0) return RF2_ERR_INVALID_ARG;
+  if (need > kScratchBytes) return RF2_ERR_WORKSPACE;  // geometry beyond the fixed maximum
+  if (qp == nullptr || kp == nullptr || idx == nullptr || cnt == nullptr) return RF2_ERR_INVALID_ARG;
+  if (!aligned16(qp) || !aligned16(kp) || !aligned16(idx) || !aligned16(cnt)) return RF2_ERR_ALIGNMENT;
+  if (kmax < kept) return RF2_ERR_INVALID_ARG;
+
+  void* base = nullptr;
+  int st = scratch_for_current_device(&base);
+  if (st != RF2_OK) return st;
+  const rf2::Geo geo = rf2::make_geo(*g);
+  const size_t means = (size_t)geo.B * geo.heads * geo.Nb * geo.D * sizeof(float);
+  unsigned char* p = static_cast<unsigned char*>(base);
+  float* qbar = reinterpret_cast<float*>(p);
+  float* kbar = reinterpret_cast<float*>(p + up(means));
+  float* scores = reinterpret_cast<float*>(p + 2 * up(means));
+
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = rf2::launch_pool(qp, kp, qbar, kbar, geo, s);
+  if (e == cudaSuccess)
+    e = rf2::launch_scores(qbar, kbar, scores, geo, (float)(1.0 / sqrt((double)geo.D)), s);
+  if (e == cudaSuccess)
+    e = rf2::launch_topk(scores, idx, cnt, kmax, kept, sink ? geo.nbh * geo.nbw : 0, geo, s);
+  if (e != cudaSuccess) return RF2_ERR_CUDA;
+  if (flags & RF2_CHECKED) {
+    if (cudaStreamSynchronize(s) != cudaSuccess) return RF2_ERR_CUDA;
+  }
+  return RF2_OK;
+}

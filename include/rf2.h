@@ -109,6 +109,34 @@ int rf2_predict_mask(const void* qp, const void* kp, const rf2_geom* g, double s
                      int sink, unsigned flags, int32_t* idx, int32_t* cnt, int kmax,
                      void* ws, size_t ws_bytes, void* stream);
 
+/* Size of the fixed device scratch of rf2_predict_mask_noalloc (16 MiB). */
+#define RF2_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* rf2_predict_mask_noalloc - rf2_predict_mask for callers that cannot allocate device
+ * memory.  The pages have no counterpart: this is a deployment variant, not a step of
+ * the method.  Some callers may not call cudaMalloc at all (code inside a framework that
+ * owns every device allocation, or a plug-in that must not allocate after start-up), so
+ * they cannot supply the `ws` scratch.  This call computes exactly what rf2_predict_mask
+ * computes, with its scratch taken from a fixed file-scope device array of
+ * RF2_NOALLOC_SCRATCH_BYTES instead; it allocates nothing.
+ *   Arguments: as rf2_predict_mask, without ws/ws_bytes.  The caller still owns qp, kp,
+ *   idx and cnt.
+ *   Limit: the geometry's rf2_workspace_size(g, sparsity, sink, flags, 0) must not exceed
+ *   RF2_NOALLOC_SCRATCH_BYTES, else the call returns RF2_ERR_WORKSPACE and launches
+ *   nothing.  (The tiny, 480p and image-edit shapes fit; the 720p and long-video ones do
+ *   not.)
+ *   Set-up: the first call on a device looks up the array's device address with that
+ *   device current (cudaGetSymbolAddress); make that first call before any stream
+ *   capture.
+ *   Sharing: the array exists on every GPU that loads the library until the process
+ *   exits, and all calls on a device share it.  Each call writes all the scratch it reads
+ *   before reading it, so nothing needs clearing; calls that overlap on the GPU (other
+ *   streams or host threads on the same device) race and must be serialised.
+ * Errors: as rf2_predict_mask. */
+int rf2_predict_mask_noalloc(const void* qp, const void* kp, const rf2_geom* g,
+                             double sparsity, int sink, unsigned flags, int32_t* idx,
+                             int32_t* cnt, int kmax, void* stream);
+
 /* rf2_sparse_attn - block-sparse attention over the kept blocks (mlsanity index page,
  * title "block-wise sparse attention"; Abstract: skipping the computation of
  * insignificant tokens).  For each (b, head, query block i):
