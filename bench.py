@@ -43,6 +43,8 @@ def _args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--heads", type=int, default=None,
+                   help="override the head count (smaller captures for profiling)")
     return p.parse_args()
 
 
@@ -182,6 +184,10 @@ def main():
     from rf2_inputs import WORKLOADS
 
     wl = WORKLOADS[a.workload]
+    if a.heads is not None:
+        import dataclasses
+
+        wl = dataclasses.replace(wl, heads=a.heads)
     sparsity = wl.sparsity if a.sparsity is None else a.sparsity
     metric = "ms/call and dense-equiv TFLOP/s at 80% sparsity, Wan-720p-shaped attention"
     unit = "dense-equiv TFLOP/s"

@@ -7,15 +7,17 @@
 //
 // One CTA per (query block, head, batch); query tile of 128 rows (a 64-token block uses
 // the first 64).  Warp roles (192 threads):
-//   warps 0-3  softmax: thread r owns query row r = TMEM lane r; reads S from TMEM,
-//              online softmax in fp32 (exp2 domain), writes P (bf16) to shared memory in
-//              the 128-byte-swizzled K-major layout, rescales O in TMEM when the running
-//              max grows by more than 2^8, and runs the epilogue (O / l -> bf16 -> HBM).
+//   warps 0-3  softmax: thread r owns query row r = TMEM lane r.  Reads the S row from
+//              TMEM in one load, online softmax in fp32 (exp2 domain), writes P (bf16
+//              pairs) back into the same TMEM columns, rescales O in TMEM when the
+//              running max grows by more than 2^8, and runs the epilogue.
 //   warp 4     TMA producer: Q once, then K_j and V_j of each kept block j through two
-//              independent 2-stage rings.
-//   warp 5     MMA issuer: S_i = Q K_i^T into one of two TMEM S buffers (SS MMA, K-major
-//              operands), then O += P_{i-1} V_{i-1} (V read MN-major) one step behind, so
-//              the tensor core computes S_{i+1} while the softmax works on S_i.
+//              independent 2-stage shared-memory rings.
+//   warp 5     MMA issuer: S_i = Q K_i^T (both operands from shared memory, K-major) into
+//              one of three TMEM S/P buffers, then O += P_{i-1} V_{i-1} with P read from
+//              TMEM and V from shared memory (MN-major), one step behind, so the tensor
+//              core computes S_{i+1} while the softmax works on S_i.
+// TMEM: three 128-column S/P buffers and the 128-column O accumulator (512 columns).
 // Every mbarrier wait is bounded in time; on expiry the CTA raises a timeout status,
 // stops issuing work, drains what it issued and returns.
 #include <cuda.h>
@@ -30,8 +32,9 @@ constexpr int kBM = 128;            // query rows per tile (TMEM lanes)
 constexpr int kThreads = 192;
 constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
+constexpr int kSBufs = 3;           // S/P buffers in TMEM
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256;
+constexpr uint32_t kTmemO = 384;    // S/P buffer b at column 128*b
 constexpr uint64_t kWaitLimitNs = 500ull * 1000ull * 1000ull;  // 0.5 s per wait
 
 template <int D, int BLK>
@@ -39,14 +42,12 @@ struct Cfg {
   static constexpr int kAtomsD = D / 64;       // 128-byte column atoms of a [rows, D] tile
   static constexpr int kQBytes = kBM * D * 2;
   static constexpr int kKVBytes = BLK * D * 2;
-  static constexpr int kPBytes = kBM * BLK * 2;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + 2 * kKVBytes;
-  static constexpr int kOffP = kOffV + 2 * kKVBytes;
-  static constexpr int kOffList = kOffP + kPBytes;     // int32[1024] compacted kept list
-  static constexpr int kOffBar = kOffList + 4096;      // mbarriers
-  static constexpr int kOffMisc = kOffBar + 256;       // tmem slot, counts, flags
+  static constexpr int kOffList = kOffV + 2 * kKVBytes;  // int32[1024] compacted kept list
+  static constexpr int kOffBar = kOffList + 4096;        // mbarriers
+  static constexpr int kOffMisc = kOffBar + 256;         // tmem slot, counts, flags
   static constexpr int kUsed = kOffMisc + 64;
   // Requested dynamic smem: 1 KB alignment slack; at least 116 KB so that at most one
   // CTA is resident per SM (each CTA allocates all 512 TMEM columns).
@@ -56,16 +57,16 @@ struct Cfg {
 // Barrier slots (8 bytes each) at kOffBar.
 enum : int {
   BAR_Q = 0,
-  BAR_KFULL = 1,   // +stage
-  BAR_KEMPTY = 3,  // +stage
-  BAR_VFULL = 5,   // +stage
-  BAR_VEMPTY = 7,  // +stage
-  BAR_SFULL = 9,   // +buffer
-  BAR_SFREE = 11,  // +buffer
-  BAR_PFULL = 13,
-  BAR_ORDY = 14,
-  BAR_DONE = 15,
-  BAR_COUNT = 16
+  BAR_KFULL = 1,    // +stage (2)
+  BAR_KEMPTY = 3,   // +stage (2)
+  BAR_VFULL = 5,    // +stage (2)
+  BAR_VEMPTY = 7,   // +stage (2)
+  BAR_SFULL = 9,    // +buffer (3): S_i computed
+  BAR_PFULL = 12,   // +buffer (3): P_i written to TMEM
+  BAR_SFREE = 15,   // +buffer (3): P_i V_i completed, buffer reusable
+  BAR_ORDY = 18,    // every P_i V_i completed (O stable)
+  BAR_DONE = 19,
+  BAR_COUNT = 20
 };
 
 struct Misc {
@@ -87,8 +88,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = ptx::smem_u32(smem);
-  const uint32_t sQ = sbase + C::kOffQ, sK = sbase + C::kOffK, sV = sbase + C::kOffV,
-                 sP = sbase + C::kOffP;
+  const uint32_t sQ = sbase + C::kOffQ, sK = sbase + C::kOffK, sV = sbase + C::kOffV;
   int* list_s = reinterpret_cast<int*>(smem + C::kOffList);
   const uint32_t bar0 = sbase + C::kOffBar;
   auto bar = [&](int k) { return bar0 + 8u * (uint32_t)k; };
@@ -116,10 +116,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(bar(BAR_KEMPTY + s), 1);
       ptx::mbar_init(bar(BAR_VFULL + s), 1);
       ptx::mbar_init(bar(BAR_VEMPTY + s), 1);
-      ptx::mbar_init(bar(BAR_SFULL + s), 1);
-      ptx::mbar_init(bar(BAR_SFREE + s), 4);
     }
-    ptx::mbar_init(bar(BAR_PFULL), 4);
+    for (int s = 0; s < kSBufs; ++s) {
+      ptx::mbar_init(bar(BAR_SFULL + s), 1);
+      ptx::mbar_init(bar(BAR_PFULL + s), 4);
+      ptx::mbar_init(bar(BAR_SFREE + s), 1);
+    }
     ptx::mbar_init(bar(BAR_ORDY), 1);
     ptx::mbar_init(bar(BAR_DONE), 1);
     misc->abort = 0;
@@ -206,43 +208,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_after();
       auto issue_pv = [&](int i) -> bool {
         const int s = i & 1;
-        if (!ptx::mbar_wait(bar(BAR_PFULL), i & 1, abort_flag, status, kWaitLimitNs,
-                            kStatusTimeout))
+        const int pb = i % kSBufs;
+        if (!ptx::mbar_wait(bar(BAR_PFULL + pb), (i / kSBufs) & 1, abort_flag, status,
+                            kWaitLimitNs, kStatusTimeout))
           return false;
         if (!ptx::mbar_wait(bar(BAR_VFULL + s), (i >> 1) & 1, abort_flag, status, kWaitLimitNs,
                             kStatusTimeout))
           return false;
         ptx::tc_fence_after();
         const uint32_t vs = sV + s * C::kKVBytes;
+        const uint32_t pt = tmem + (uint32_t)(128 * pb);
 #pragma unroll
         for (int kk = 0; kk < BLK / 16; ++kk) {
-          // A = P [128 x BLK] K-major (keys contiguous); step kk = 16 keys = 32 bytes
-          const uint64_t ad =
-              ptx::smem_desc_sw128(sP + (kk >> 2) * (kBM * 128) + (kk & 3) * 32, 16, 1024);
+          // A = P [128 x BLK] in TMEM: 16 keys = 8 columns of bf16 pairs.
           // B = V [BLK keys x D] read as N x K MN-major: 16 keys = 16 rows of 128 bytes;
           // the D atoms (64 columns each) are BLK*128 bytes apart.
           const uint64_t bd = ptx::smem_desc_sw128(vs + kk * (16 * 128), BLK * 128, 1024);
-          ptx::mma_f16_ss(tmem + kTmemO, ad, bd, idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+          ptx::mma_f16_ts(tmem + kTmemO, pt + kk * 8, bd, idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
         }
         ptx::mma_commit(bar(BAR_ORDY));
         ptx::mma_commit(bar(BAR_VEMPTY + s));
+        ptx::mma_commit(bar(BAR_SFREE + pb));
         return true;
       };
       for (int i = 0; ok && i < n; ++i) {
         const int s = i & 1;
+        const int sb = i % kSBufs;
         if (!ptx::mbar_wait(bar(BAR_KFULL + s), (i >> 1) & 1, abort_flag, status, kWaitLimitNs,
                             kStatusTimeout)) {
           ok = false;
           break;
         }
-        if (i >= 2 && !ptx::mbar_wait(bar(BAR_SFREE + s), ((i >> 1) & 1) ^ 1, abort_flag, status,
-                                      kWaitLimitNs, kStatusTimeout)) {
+        // S/P buffer sb last held P_{i-3}: reusable once P_{i-3} V_{i-3} has completed.
+        if (i >= kSBufs && !ptx::mbar_wait(bar(BAR_SFREE + sb), ((i / kSBufs) - 1) & 1, abort_flag,
+                                           status, kWaitLimitNs, kStatusTimeout)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
         const uint32_t ks = sK + s * C::kKVBytes;
-        const uint32_t dS = tmem + (s ? kTmemS1 : kTmemS0);
+        const uint32_t dS = tmem + (uint32_t)(128 * sb);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk & 3) * 32;  // 16 columns = 32 bytes inside an atom
@@ -250,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = ptx::smem_desc_sw128(ks + (kk >> 2) * (BLK * 128) + koff, 16, 1024);
           ptx::mma_f16_ss(dS, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
-        ptx::mma_commit(bar(BAR_SFULL + s));
+        ptx::mma_commit(bar(BAR_SFULL + sb));
         ptx::mma_commit(bar(BAR_KEMPTY + s));
         if (i >= 1 && !issue_pv(i - 1)) {
           ok = false;
@@ -269,32 +274,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       float l_run = 0.f;
       bool ok = true;
       for (int i = 0; i < n; ++i) {
-        const int s = i & 1;
+        const int sb = i % kSBufs;
         const int j = list_s[i];
+        const uint32_t srow = tmem + lane_base + (uint32_t)(128 * sb);
         // Waits are per thread; giving up is decided for the whole warp so that the
         // warp-wide tcgen05 and shuffle operations below stay converged.
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(BAR_SFULL + s), (i >> 1) & 1, abort_flag,
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(BAR_SFULL + sb), (i / kSBufs) & 1, abort_flag,
                                                      status, kWaitLimitNs, kStatusTimeout))) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
         float x[BLK];
+        {
+          // the whole S row in one TMEM load (one round trip)
+          uint32_t t[BLK];
+          if constexpr (BLK == 128)
+            ptx::tmem_ld32x128(srow, t);
+          else
+            ptx::tmem_ld32x64(srow, t);
 #pragma unroll
-        for (int c = 0; c < BLK / 32; ++c) {
-          uint32_t t[32];
-          ptx::tmem_ld32(tmem + lane_base + (s ? kTmemS1 : kTmemS0) + c * 32, t);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(t[e]);
+          for (int c = 0; c < BLK; ++c) x[c] = __uint_as_float(t[c]);
         }
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(BAR_SFREE + s));
         // Pad keys of a partial window get -inf; validity is per column, the same for
         // every row, so each lane evaluates 1/32 of the columns and the warp shares bits.
         int nt, nh, nw;
         block_extent(g, j, nt, nh, nw);
-        float mx = -INFINITY;
         if (nt < g.wt || nh < g.wh || nw < g.ww) {
           uint32_t vm[BLK / 32];
           const int whw = g.wh * g.ww;
@@ -308,21 +313,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             vm[q] = __ballot_sync(0xffffffffu, dt < nt && dh < nh && dw < nw);
           }
 #pragma unroll
-          for (int c = 0; c < BLK; ++c) {
-            const bool v = (vm[c >> 5] >> (c & 31)) & 1u;
-            x[c] = v ? x[c] * scale_log2 : -INFINITY;
-            mx = fmaxf(mx, x[c]);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < BLK; ++c) {
-            x[c] *= scale_log2;
-            mx = fmaxf(mx, x[c]);
-          }
+          for (int c = 0; c < BLK; ++c)
+            if (!((vm[c >> 5] >> (c & 31)) & 1u)) x[c] = -INFINITY;
         }
-        // Running max: only moved when it grows by more than 2^8 (in exp2 units), so
-        // P <= 256 and O needs rescaling rarely; the final O / l is unchanged by this.
-        const float m_new = fmaxf(m_run, mx);
+        // Row max of the raw scores (scale > 0 commutes with max) over 8 independent
+        // chains, so the reduction is not one long dependency chain.
+        float mx8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx8[e] = x[e];
+#pragma unroll
+        for (int c = 8; c < BLK; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        // Running max in exp2 units: only moved when it grows by more than 8, so P <= 2^8
+        // and O needs rescaling rarely; the final O / l is unchanged by this.
+        const float m_new = fmaxf(m_run, mx * scale_log2);
         const bool grow = m_new > m_run + 8.0f;  // always true on the first block
         float alpha = 1.0f;
         if (grow) {
@@ -330,15 +335,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           l_run *= alpha;
           m_run = m_new;
         }
-        // P buffer is free and O is stable once P_{i-1} V_{i-1} has completed.
-        if (i >= 1 && !__all_sync(0xffffffffu, ptx::mbar_wait(bar(BAR_ORDY), (i - 1) & 1, abort_flag,
-                                                             status, kWaitLimitNs, kStatusTimeout))) {
-          ok = false;
-          break;
-        }
         if (i >= 1 && __any_sync(0xffffffffu, grow)) {
-          // tcgen05.ld/st are warp-wide: the warp rescales its 32 rows of O together,
-          // rows that did not grow with alpha = 1.
+          // O is stable once P_{i-1} V_{i-1} has completed.  S_i completing implies that
+          // P_{i-2} V_{i-2} has (a commit covers every earlier MMA), and P_i V_i cannot
+          // start before this warp publishes P_i, so BAR_ORDY is in phase i-1 or i here
+          // and its parity wait is unambiguous.  tcgen05.ld/st are
+          // warp-wide: the warp rescales its 32 rows of O together, rows that did not
+          // grow with alpha = 1.
+          if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(BAR_ORDY), (i - 1) & 1, abort_flag,
+                                                       status, kWaitLimitNs, kStatusTimeout))) {
+            ok = false;
+            break;
+          }
           ptx::tc_fence_after();
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
@@ -348,35 +356,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < 32; ++e) t[e] = __float_as_uint(__uint_as_float(t[e]) * alpha);
             ptx::tmem_st32(tmem + lane_base + kTmemO + c * 32, t);
           }
-          ptx::tmem_wait_st();
         }
-        // P = exp2(x - m_run), rounded to bf16, to shared memory (128B-swizzled, K-major).
-        const uint32_t prow = sP + (uint32_t)r * 128u;
+        // P = exp2(s * scale_log2 - m_run): one FFMA and one ex2 per element, rounded to
+        // bf16 pairs and written over the first BLK/2 columns of this S buffer (the A
+        // operand of P V); the row sum uses 8 independent accumulators.
+        const float neg_m = -m_run;
+        float ls[8];
 #pragma unroll
-        for (int q = 0; q < BLK / 8; ++q) {
-          uint32_t pk[4];
+        for (int e = 0; e < 8; ++e) ls[e] = 0.f;
+        uint32_t pk[BLK / 2];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p0 = ptx::ex2(x[q * 8 + 2 * e] - m_run);
-            const float p1 = ptx::ex2(x[q * 8 + 2 * e + 1] - m_run);
-            l_run += p0 + p1;
-            pk[e] = ptx::pack_bf16(p0, p1);
-          }
-          const uint32_t atom = (uint32_t)(q >> 3);
-          const uint32_t chunk = (uint32_t)((q & 7) ^ (r & 7));
-          const uint32_t addr = prow + atom * (kBM * 128) + chunk * 16;
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[0]),
-                       "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
-                       : "memory");
+        for (int c2 = 0; c2 < BLK / 2; ++c2) {
+          const float p0 = ptx::ex2(fmaf(x[2 * c2], scale_log2, neg_m));
+          const float p1 = ptx::ex2(fmaf(x[2 * c2 + 1], scale_log2, neg_m));
+          ls[(2 * c2) & 7] += p0;
+          ls[(2 * c2 + 1) & 7] += p1;
+          pk[c2] = ptx::pack_bf16(p0, p1);
         }
-        ptx::fence_proxy_async_smem();
+        if constexpr (BLK == 128) {
+          ptx::tmem_st32x64(srow, pk);
+        } else {
+          ptx::tmem_st32(srow, pk);
+        }
+        ptx::tmem_wait_st();
+        l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(BAR_PFULL));
+        if (lane == 0) ptx::mbar_arrive(bar(BAR_PFULL + sb));
       }
       // ---------------------------------------------------------- epilogue
-      if (ok && __all_sync(0xffffffffu, ptx::mbar_wait(bar(BAR_ORDY), (n - 1) & 1, abort_flag,
-                                                       status, kWaitLimitNs, kStatusTimeout))) {
+      // BAR_DONE fires once every MMA of the CTA has completed (the softmax skips most
+      // BAR_ORDY phases, so a parity wait there could alias an older phase).
+      if (ok && __all_sync(0xffffffffu, ptx::mbar_wait(bar(BAR_DONE), 0, abort_flag, status,
+                                                       kWaitLimitNs, kStatusTimeout))) {
         ptx::tc_fence_after();
         const float inv = l_run > 0.f ? 1.0f / l_run : 0.f;
         __nv_bfloat16* orow =
@@ -416,6 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 }  // namespace rf2
+
 
 namespace rf2 {
 namespace {

@@ -223,7 +223,7 @@ int rf2_sparse_attn(const void* qp, const void* kp, const void* vp, const int32_
   int st = check_geom(g);
   if (st != RF2_OK) return st;
   if (qp == nullptr || kp == nullptr || vp == nullptr || idx == nullptr || cnt == nullptr ||
-      op == nullptr || kmax < 1 || !isfinite(scale))
+      op == nullptr || kmax < 1 || !isfinite(scale) || scale < 0.f)
     return RF2_ERR_INVALID_ARG;
   if (!aligned16(qp) || !aligned16(kp) || !aligned16(vp) || !aligned16(op) ||
       ((uintptr_t)idx & 3u) || ((uintptr_t)cnt & 3u) || ((uintptr_t)status & 3u))
@@ -243,7 +243,8 @@ int rf2_attention(const void* q, const void* k, const void* v, const rf2_geom* g
                   unsigned flags, void* stream) {
   int st = check_geom(g);
   if (st != RF2_OK) return st;
-  if (!(sparsity >= 0.0 && sparsity <= 1.0) || !isfinite(scale)) return RF2_ERR_INVALID_ARG;
+  if (!(sparsity >= 0.0 && sparsity <= 1.0) || !isfinite(scale) || scale < 0.f)
+    return RF2_ERR_INVALID_ARG;
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return RF2_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
       ((uintptr_t)idx_out & 3u))

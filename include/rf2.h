@@ -144,7 +144,8 @@ int rf2_predict_mask_noalloc(const void* qp, const void* kp, const rf2_geom* g,
  *   S = idx[b, head, i, 0..cnt-1]; M = -inf on pad keys, 0 elsewhere.
  *   qp, kp, vp : [B, Npad, heads, D] bf16 (read).   op : [B, Npad, heads, D] bf16
  *   (written; pad query rows are written too, with values of no meaning).
- *   scale : softmax scale; 0 means 1/sqrt(D).  Softmax statistics and the accumulator
+ *   scale : softmax scale, > 0; 0 means 1/sqrt(D) (negative: RF2_ERR_INVALID_ARG).
+ *   Softmax statistics and the accumulator
  *   are fp32; P is rounded to bf16 for the P.V product.
  *   status : optional device int32 (may be NULL); when given it must be zero on entry
  *   and receives RF2_ERR_BAD_INDEX / RF2_ERR_TIMEOUT if the kernel detects one
