@@ -6,7 +6,7 @@
 //            HBM-bound streaming reduction over the permuted Q and K.
 //   scores : s[b, head, i, j] = qbar_i . kbar_j * scale, an fp32 register-tiled product.
 //   topk   : per row, the sink blocks plus the m best other blocks (ties to the lower
-//            id) as an ascending list; one warp per row, exact bitwise radix select.
+//            id) as an ascending list; one warp per row, exact bitwise search.
 #include "rf2_common.cuh"
 
 namespace rf2 {
@@ -97,12 +97,20 @@ __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ q
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
   for (int d0 = 0; d0 < g.D; d0 += kSSlab) {
-    // load: 64 rows x 32 d for each operand; thread loads 8 elements of each
-    for (int e = tid; e < kSTile * kSSlab; e += 256) {
-      int r = e / kSSlab, d = e - r * kSSlab;
-      int gi = i0 + r, gj = j0 + r;
-      qs[d][r] = gi < g.Nb ? qb[(long long)gi * g.D + d0 + d] : 0.f;
-      ks[d][r] = gj < g.Nb ? kb[(long long)gj * g.D + d0 + d] : 0.f;
+    // Slab fill: 64 rows x 32 d of each operand as 512 float4 per operand.  Within a
+    // warp consecutive threads take consecutive rows of the same 4 d, so the transposed
+    // (d-major) shared-memory stores hit 32 different banks.
+#pragma unroll
+    for (int it = 0; it < (kSTile * kSSlab / 4) / 256; ++it) {
+      const int f = tid + 256 * it;
+      const int r = f % kSTile, d4 = f / kSTile;
+      const int gi = i0 + r, gj = j0 + r;
+      float4 qv = gi < g.Nb ? *reinterpret_cast<const float4*>(qb + (long long)gi * g.D + d0 + 4 * d4)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 kv = gj < g.Nb ? *reinterpret_cast<const float4*>(kb + (long long)gj * g.D + d0 + 4 * d4)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+      qs[4 * d4 + 0][r] = qv.x; qs[4 * d4 + 1][r] = qv.y; qs[4 * d4 + 2][r] = qv.z; qs[4 * d4 + 3][r] = qv.w;
+      ks[4 * d4 + 0][r] = kv.x; ks[4 * d4 + 1][r] = kv.y; ks[4 * d4 + 2][r] = kv.z; ks[4 * d4 + 3][r] = kv.w;
     }
     __syncthreads();
 #pragma unroll 8
@@ -132,10 +140,11 @@ __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ q
 }
 
 // ------------------------------------------------------------------------------- top-k
-// One warp per (b, head, i) row.  Scores map to order-preserving uint32 keys; the m-th
-// largest candidate key is found by a 32-step bitwise search (exact); candidates above
-// it are kept, and equal ones in ascending block order until m are kept.  The output
-// list (sink blocks and kept candidates) is emitted in ascending order with ballots.
+// One warp per (b, head, i) row.  Scores map to order-preserving uint32 keys (every real
+// key is > 0; 0 marks a non-candidate).  The m-th largest candidate key is found exactly
+// by a 32-step bitwise search with warp-wide counts; candidates above it are kept, and
+// equal ones in ascending block order until m are kept.  The output list (sink blocks and kept candidates) is
+// emitted in ascending order with ballots.
 constexpr int kTopkWarps = 8;
 constexpr int kMaxPerLane = 32;  // Nb <= 1024
 
@@ -144,69 +153,76 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+template <int KPL>
+__device__ __forceinline__ void topk_row(const float* __restrict__ sr, int32_t* __restrict__ out,
+                                         int32_t* __restrict__ cnt_out, int Nb, int kmax, int kept,
+                                         int nsink, int lane) {
+  uint32_t key[KPL];
+#pragma unroll
+  for (int k = 0; k < KPL; ++k) {
+    const int j = k * 32 + lane;
+    key[k] = (j < Nb && j >= nsink) ? order_key(__ldg(sr + j)) : 0u;
+  }
+  const int m = kept - nsink;
+  const int ncand = Nb - nsink;
+  uint32_t thr = 0;   // the m-th largest candidate key
+  int take_eq = 0;    // how many keys equal to thr are kept (lowest ids first)
+  if (m > 0 && m < ncand) {
+    // Bitwise search from the most significant bit: the largest t with
+    // #{key >= t} >= m is the m-th largest key.
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t t = thr | (1u << bit);
+      int c = 0;
+#pragma unroll
+      for (int k = 0; k < KPL; ++k) c += key[k] >= t;
+      if ((int)__reduce_add_sync(0xffffffffu, (uint32_t)c) >= m) thr = t;
+    }
+    int above = 0;
+#pragma unroll
+    for (int k = 0; k < KPL; ++k) above += key[k] > thr;
+    take_eq = m - (int)__reduce_add_sync(0xffffffffu, (uint32_t)above);
+  } else if (m >= ncand) {
+    thr = 1u;  // every candidate
+  } else {
+    thr = 0xffffffffu;  // m == 0: none
+  }
+  int pos = 0;
+  int eq_taken = 0;
+  const bool all = m >= ncand;
+  const bool some = m > 0 && m < ncand;
+#pragma unroll
+  for (int k = 0; k < KPL; ++k) {
+    if (k * 32 >= Nb) break;
+    const int j = k * 32 + lane;
+    const bool in_range = j < Nb;
+    const bool is_sink = in_range && j < nsink;
+    const bool above = in_range && !is_sink && (all ? key[k] != 0u : key[k] > thr);
+    const bool eq = in_range && !is_sink && some && key[k] == thr;
+    const uint32_t eqmask = __ballot_sync(0xffffffffu, eq);
+    const int eq_rank = eq_taken + __popc(eqmask & ((1u << lane) - 1u));
+    const bool take = is_sink || above || (eq && eq_rank < take_eq);
+    eq_taken += __popc(eqmask);
+    const uint32_t tmask = __ballot_sync(0xffffffffu, take);
+    const int p = pos + __popc(tmask & ((1u << lane) - 1u));
+    if (take && p < kmax) out[p] = j;
+    pos += __popc(tmask);
+  }
+  for (int p = pos + lane; p < kmax; p += 32) out[p] = -1;
+  if (lane == 0) *cnt_out = pos;
+}
+
+template <int KPL>
 __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __restrict__ s,
                                                                int32_t* __restrict__ idx,
                                                                int32_t* __restrict__ cnt,
                                                                int Nb, long long rows, int kmax,
                                                                int kept, int nsink) {
   const int lane = threadIdx.x & 31;
-  const long long row = (long long)blockIdx.x * kTopkWarps + (threadIdx.x >> 5);
+  const int w = threadIdx.x >> 5;
+  const long long row = (long long)blockIdx.x * kTopkWarps + w;
   if (row >= rows) return;
-  const float* sr = s + row * Nb;
-  // keys of candidates; 0 marks "not a candidate" (every real key is > 0)
-  uint32_t key[kMaxPerLane];
-#pragma unroll
-  for (int k = 0; k < kMaxPerLane; ++k) {
-    int j = k * 32 + lane;
-    key[k] = (j < Nb && j >= nsink) ? order_key(sr[j]) : 0u;
-  }
-  const int m = kept - nsink;
-  const int ncand = Nb - nsink;
-  uint32_t thr = 0;  // keys >= thr are in; the last `need_eq` keys equal to thr by id
-  int take_eq = 0;
-  if (m > 0 && m < ncand) {
-    for (int bit = 31; bit >= 0; --bit) {
-      uint32_t t = thr | (1u << bit);
-      int c = 0;
-#pragma unroll
-      for (int k = 0; k < kMaxPerLane; ++k) c += key[k] >= t;
-      c = __reduce_add_sync(0xffffffffu, c);
-      if (c >= m) thr = t;
-    }
-    int above = 0;
-#pragma unroll
-    for (int k = 0; k < kMaxPerLane; ++k) above += key[k] > thr;
-    above = __reduce_add_sync(0xffffffffu, above);
-    take_eq = m - above;
-  } else if (m >= ncand) {
-    thr = 1u;  // every candidate (all real keys are >= 1)
-    take_eq = 0;
-  } else {
-    thr = 0xffffffffu;  // none: m == 0
-    take_eq = 0;
-  }
-  int32_t* out = idx + row * kmax;
-  int pos = 0;
-  int eq_taken = 0;
-#pragma unroll
-  for (int k = 0; k < kMaxPerLane; ++k) {
-    if (k * 32 >= Nb) break;
-    int j = k * 32 + lane;
-    bool in_range = j < Nb;
-    bool is_sink = in_range && j < nsink;
-    bool above = in_range && !is_sink && (m >= ncand ? key[k] != 0u : key[k] > thr);
-    bool eq = in_range && !is_sink && m < ncand && m > 0 && key[k] == thr;
-    uint32_t eqmask = __ballot_sync(0xffffffffu, eq);
-    int eq_rank = eq_taken + __popc(eqmask & ((1u << lane) - 1u));
-    bool take = is_sink || above || (eq && eq_rank < take_eq);
-    eq_taken += __popc(eqmask);
-    uint32_t tmask = __ballot_sync(0xffffffffu, take);
-    int p = pos + __popc(tmask & ((1u << lane) - 1u));
-    if (take && p < kmax) out[p] = j;
-    pos += __popc(tmask);
-  }
-  for (int p = pos + lane; p < kmax; p += 32) out[p] = -1;
-  if (lane == 0) cnt[row] = pos;
+  topk_row<KPL>(s + row * Nb, idx + row * kmax, cnt + row, Nb, kmax, kept, nsink, lane);
 }
 
 }  // namespace
@@ -232,8 +248,15 @@ cudaError_t launch_topk(const float* scores, int32_t* idx, int32_t* cnt, int kma
   if (g.Nb > kMaxPerLane * 32) return cudaErrorNotSupported;
   long long rows = (long long)g.B * g.heads * g.Nb;
   long long grid = (rows + kTopkWarps - 1) / kTopkWarps;
-  topk_kernel<<<(unsigned)grid, kTopkWarps * 32, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax,
-                                                         kept, nsink);
+  // keys per lane: the smallest instance that covers Nb
+  if (g.Nb <= 256)
+    topk_kernel<8><<<(unsigned)grid, kTopkWarps * 32, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
+  else if (g.Nb <= 512)
+    topk_kernel<16><<<(unsigned)grid, kTopkWarps * 32, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
+  else if (g.Nb <= 768)
+    topk_kernel<24><<<(unsigned)grid, kTopkWarps * 32, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
+  else
+    topk_kernel<32><<<(unsigned)grid, kTopkWarps * 32, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
   return cudaGetLastError();
 }
 
