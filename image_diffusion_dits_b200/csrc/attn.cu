@@ -6,18 +6,24 @@
 //   M = -inf on pad keys (partial windows at the high end of an axis).
 //
 // One CTA per (query block, head, batch); query tile of 128 rows (a 64-token block uses
-// the first 64).  Warp roles (192 threads):
-//   warps 0-3  softmax: thread r owns query row r = TMEM lane r.  Reads the S row from
-//              TMEM in one load, online softmax in fp32 (exp2 domain), writes P (bf16
-//              pairs) back into the same TMEM columns, rescales O in TMEM when the
-//              running max grows by more than 2^8, and runs the epilogue.
-//   warp 4     TMA producer: Q once, then K_j and V_j of each kept block j through two
-//              independent 2-stage shared-memory rings.
-//   warp 5     MMA issuer: S_i = Q K_i^T (both operands from shared memory, K-major) into
-//              one of three TMEM S/P buffers, then O += P_{i-1} V_{i-1} with P read from
-//              TMEM and V from shared memory (MN-major), one step behind, so the tensor
-//              core computes S_{i+1} while the softmax works on S_i.
-// TMEM: three 128-column S/P buffers and the 128-column O accumulator (512 columns).
+// the first 64).  The kept blocks of the row are split into two streams, even and odd
+// positions of the list; each stream has its own softmax warpgroup, running max, row
+// sum, S/P buffer and O accumulator in TMEM, and the two partial results are merged in
+// the epilogue (softmax over the union = the two partial softmaxes rescaled to a common
+// max).  The streams run concurrently, so one warpgroup's TMEM round trips and
+// exponentials overlap the other's, and the tensor core always has a tile of one
+// stream to work on while the other stream's softmax runs.
+// Warp roles (352 threads):
+//   warps 0-3  softmax of stream 0, warps 4-7 softmax of stream 1: thread r owns query
+//              row r = TMEM lane r.  Reads the S row in one TMEM load, online softmax in
+//              fp32 (exp2 domain), writes P (bf16 pairs) over the S columns, rescales its
+//              O when its running max grows by more than 2^8.
+//   warp 8     TMA producer of Q (once) and of K_j for each kept block j (3-stage ring).
+//   warp 9     MMA issuer: S_i = Q K_i^T (SS, K-major) into the S/P buffer of stream i%2,
+//              O_{i%2} += P_i V_i (P from TMEM, V MN-major from shared memory), then
+//              S_{i+2} into the same buffer right behind it (MMAs execute in issue order).
+//   warp 10    TMA producer of V_j (2-stage ring).
+// TMEM: S/P buffers at columns 0 and 128, O accumulators at 256 and 384 (512 columns).
 // Every mbarrier wait is bounded in time; on expiry the CTA raises a timeout status,
 // stops issuing work, drains what it issued and returns.
 #include <cuda.h>
@@ -29,12 +35,15 @@ namespace rf2 {
 namespace {
 
 constexpr int kBM = 128;            // query rows per tile (TMEM lanes)
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kSBufs = 3;           // S/P buffers in TMEM
+constexpr int kSoftmaxWarps = 8;    // two warpgroups, one per stream
+constexpr int kThreads = 352;       // 8 softmax warps + K producer + MMA + V producer
+constexpr int kProducerWarp = 8;    // Q and K loads
+constexpr int kMmaWarp = 9;
+constexpr int kVProducerWarp = 10;  // V loads
+constexpr int kKStages = 3;         // K ring depth
+constexpr int kVStages = 2;         // V ring depth
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 384;    // S/P buffer b at column 128*b
+constexpr uint32_t kTmemO = 256;    // O of stream s at kTmemO + 128*s; S/P of stream s at 128*s
 constexpr uint64_t kWaitLimitNs = 500ull * 1000ull * 1000ull;  // 0.5 s per wait
 
 template <int D, int BLK>
@@ -44,9 +53,11 @@ struct Cfg {
   static constexpr int kKVBytes = BLK * D * 2;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffV = kOffK + 2 * kKVBytes;
-  static constexpr int kOffList = kOffV + 2 * kKVBytes;  // int32[1024] compacted kept list
-  static constexpr int kOffBar = kOffList + 4096;        // mbarriers
+  static constexpr int kOffV = kOffK + kKStages * kKVBytes;
+  static constexpr int kOffList = kOffV + kVStages * kKVBytes;  // int32[1024] kept list
+  static constexpr int kOffExt = kOffList + 4096;        // int32[1024] real extent per entry
+  static constexpr int kOffXch = kOffExt + 4096;         // float[2 stream][2 (m,l)][128]
+  static constexpr int kOffBar = kOffXch + 2048;         // mbarriers
   static constexpr int kOffMisc = kOffBar + 256;         // tmem slot, counts, flags
   static constexpr int kUsed = kOffMisc + 64;
   // Requested dynamic smem: 1 KB alignment slack; at least 116 KB so that at most one
@@ -57,16 +68,15 @@ struct Cfg {
 // Barrier slots (8 bytes each) at kOffBar.
 enum : int {
   BAR_Q = 0,
-  BAR_KFULL = 1,    // +stage (2)
-  BAR_KEMPTY = 3,   // +stage (2)
-  BAR_VFULL = 5,    // +stage (2)
-  BAR_VEMPTY = 7,   // +stage (2)
-  BAR_SFULL = 9,    // +buffer (3): S_i computed
-  BAR_PFULL = 12,   // +buffer (3): P_i written to TMEM
-  BAR_SFREE = 15,   // +buffer (3): P_i V_i completed, buffer reusable
-  BAR_ORDY = 18,    // every P_i V_i completed (O stable)
-  BAR_DONE = 19,
-  BAR_COUNT = 20
+  BAR_KFULL = 1,    // +stage (3)
+  BAR_KEMPTY = 4,   // +stage (3)
+  BAR_VFULL = 7,    // +stage (2)
+  BAR_VEMPTY = 9,   // +stage (2)
+  BAR_SFULL = 11,   // +stream (2): S_i of the stream computed
+  BAR_PFULL = 13,   // +stream (2): P_i of the stream written to TMEM
+  BAR_DONE = 15,    // every MMA of the CTA completed
+  BAR_XCH = 16,     // both warpgroups posted their (max, sum)
+  BAR_COUNT = 17
 };
 
 struct Misc {
@@ -111,24 +121,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid == 0) {
     ptx::mbar_init(bar(BAR_Q), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       ptx::mbar_init(bar(BAR_KFULL + s), 1);
       ptx::mbar_init(bar(BAR_KEMPTY + s), 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       ptx::mbar_init(bar(BAR_VFULL + s), 1);
       ptx::mbar_init(bar(BAR_VEMPTY + s), 1);
     }
-    for (int s = 0; s < kSBufs; ++s) {
+    for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(bar(BAR_SFULL + s), 1);
       ptx::mbar_init(bar(BAR_PFULL + s), 4);
-      ptx::mbar_init(bar(BAR_SFREE + s), 1);
     }
-    ptx::mbar_init(bar(BAR_ORDY), 1);
     ptx::mbar_init(bar(BAR_DONE), 1);
+    ptx::mbar_init(bar(BAR_XCH), kSoftmaxWarps);
     misc->abort = 0;
     ptx::fence_mbar_init();
   }
+  int* ext_s = reinterpret_cast<int*>(smem + C::kOffExt);
   if (warp == kProducerWarp) {
-    // Compact the kept list into shared memory, dropping ids outside [0, Nb).
+    // Compact the kept list into shared memory, dropping ids outside [0, Nb); with each
+    // kept block store its real extent (nt | nh << 8 | nw << 16) for the pad-key mask.
     int n_in = cnt[row];
     n_in = n_in < 0 ? 0 : (n_in > kmax ? kmax : n_in);
     n_in = n_in > 1024 ? 1024 : n_in;  // capacity of the shared-memory list
@@ -141,7 +154,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = e < n_in && j >= 0 && j < g.Nb;
       bad |= (e < n_in) && !ok;
       uint32_t m = __ballot_sync(0xffffffffu, ok);
-      if (ok) list_s[n_out + __popc(m & ((1u << lane) - 1u))] = j;
+      if (ok) {
+        int nt, nh, nw;
+        block_extent(g, j, nt, nh, nw);
+        const int pos = n_out + __popc(m & ((1u << lane) - 1u));
+        list_s[pos] = j;
+        ext_s[pos] = nt | (nh << 8) | (nw << 16);
+      }
       n_out += __popc(m);
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0 && status != nullptr)
@@ -156,49 +175,62 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (n > 0) {
     if (warp == kProducerWarp && lane == 0) {
-      // ------------------------------------------------------------ TMA producer
+      // ------------------------------------------------------------ TMA producer: Q, K
       ptx::prefetch_tmap(&tq);
       ptx::prefetch_tmap(&tk);
-      ptx::prefetch_tmap(&tv);
       ptx::mbar_arrive_expect_tx(bar(BAR_Q), C::kQBytes);
 #pragma unroll
       for (int a = 0; a < C::kAtomsD; ++a)
         ptx::tma_load_3d(sQ + a * (kBM * 128), &tq, bar(BAR_Q), a * 64, head,
                          (int)(brow0 + (long long)qblk * BLK));
-      int issued_k[2] = {-1, -1}, issued_v[2] = {-1, -1};
+      int issued[kKStages];
+#pragma unroll
+      for (int s = 0; s < kKStages; ++s) issued[s] = -1;
       for (int i = 0; i < n; ++i) {
-        const int s = i & 1;
-        const int zrow = (int)(brow0 + (long long)list_s[i] * BLK);
-        if (i >= 2 && !ptx::mbar_wait(bar(BAR_KEMPTY + s), ((i >> 1) & 1) ^ 1, abort_flag, status,
-                                      kWaitLimitNs, kStatusTimeout))
+        const int s = i % kKStages;
+        if (i >= kKStages && !ptx::mbar_wait(bar(BAR_KEMPTY + s), ((i / kKStages) - 1) & 1, abort_flag,
+                                             status, kWaitLimitNs, kStatusTimeout))
           break;
         ptx::mbar_arrive_expect_tx(bar(BAR_KFULL + s), C::kKVBytes);
+        const int zrow = (int)(brow0 + (long long)list_s[i] * BLK);
 #pragma unroll
         for (int a = 0; a < C::kAtomsD; ++a)
           ptx::tma_load_3d(sK + s * C::kKVBytes + a * (BLK * 128), &tk, bar(BAR_KFULL + s), a * 64,
                            head, zrow);
-        issued_k[s] = i;
-        if (i >= 2 && !ptx::mbar_wait(bar(BAR_VEMPTY + s), ((i >> 1) & 1) ^ 1, abort_flag, status,
-                                      kWaitLimitNs, kStatusTimeout))
-          break;
-        ptx::mbar_arrive_expect_tx(bar(BAR_VFULL + s), C::kKVBytes);
-#pragma unroll
-        for (int a = 0; a < C::kAtomsD; ++a)
-          ptx::tma_load_3d(sV + s * C::kKVBytes + a * (BLK * 128), &tv, bar(BAR_VFULL + s), a * 64,
-                           head, zrow);
-        issued_v[s] = i;
+        issued[s] = i;
       }
       if (*abort_flag) {
         // Let every copy this thread issued land before the CTA can exit.
         ptx::mbar_wait(bar(BAR_Q), 0, nullptr, nullptr, kWaitLimitNs, 0);
-        for (int s = 0; s < 2; ++s) {
-          if (issued_k[s] >= 0)
-            ptx::mbar_wait(bar(BAR_KFULL + s), (issued_k[s] >> 1) & 1, nullptr, nullptr,
+        for (int s = 0; s < kKStages; ++s)
+          if (issued[s] >= 0)
+            ptx::mbar_wait(bar(BAR_KFULL + s), (issued[s] / kKStages) & 1, nullptr, nullptr,
                            kWaitLimitNs, 0);
-          if (issued_v[s] >= 0)
-            ptx::mbar_wait(bar(BAR_VFULL + s), (issued_v[s] >> 1) & 1, nullptr, nullptr,
+      }
+    } else if (warp == kVProducerWarp && lane == 0) {
+      // ------------------------------------------------------------ TMA producer: V
+      ptx::prefetch_tmap(&tv);
+      int issued[kVStages];
+#pragma unroll
+      for (int s = 0; s < kVStages; ++s) issued[s] = -1;
+      for (int i = 0; i < n; ++i) {
+        const int s = i % kVStages;
+        if (i >= kVStages && !ptx::mbar_wait(bar(BAR_VEMPTY + s), ((i / kVStages) - 1) & 1, abort_flag,
+                                             status, kWaitLimitNs, kStatusTimeout))
+          break;
+        ptx::mbar_arrive_expect_tx(bar(BAR_VFULL + s), C::kKVBytes);
+        const int zrow = (int)(brow0 + (long long)list_s[i] * BLK);
+#pragma unroll
+        for (int a = 0; a < C::kAtomsD; ++a)
+          ptx::tma_load_3d(sV + s * C::kKVBytes + a * (BLK * 128), &tv, bar(BAR_VFULL + s), a * 64,
+                           head, zrow);
+        issued[s] = i;
+      }
+      if (*abort_flag) {
+        for (int s = 0; s < kVStages; ++s)
+          if (issued[s] >= 0)
+            ptx::mbar_wait(bar(BAR_VFULL + s), (issued[s] / kVStages) & 1, nullptr, nullptr,
                            kWaitLimitNs, 0);
-        }
       }
     } else if (warp == kMmaWarp && lane == 0) {
       // ------------------------------------------------------------ MMA issuer
@@ -206,81 +238,95 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_o = ptx::idesc_bf16_f32(kBM, D, 1);
       bool ok = ptx::mbar_wait(bar(BAR_Q), 0, abort_flag, status, kWaitLimitNs, kStatusTimeout);
       ptx::tc_fence_after();
-      auto issue_pv = [&](int i) -> bool {
-        const int s = i & 1;
-        const int pb = i % kSBufs;
-        if (!ptx::mbar_wait(bar(BAR_PFULL + pb), (i / kSBufs) & 1, abort_flag, status,
+      // S_i into the S/P buffer of stream i%2.  For i >= 2 that buffer holds P_{i-2}, which
+      // P_{i-2} V_{i-2} reads; that MMA was issued before this one by this thread, and
+      // tcgen05 MMAs issued by one thread execute in issue order, so S_i is issued
+      // without waiting for it to complete (no drain of the tensor pipe per block).
+      auto issue_s = [&](int i) -> bool {
+        const int ks = i % kKStages;
+        const int st = i & 1;
+        if (!ptx::mbar_wait(bar(BAR_KFULL + ks), (i / kKStages) & 1, abort_flag, status,
                             kWaitLimitNs, kStatusTimeout))
           return false;
-        if (!ptx::mbar_wait(bar(BAR_VFULL + s), (i >> 1) & 1, abort_flag, status, kWaitLimitNs,
+        ptx::tc_fence_after();
+        const uint32_t kb = sK + ks * C::kKVBytes;
+        const uint32_t dS = tmem + (uint32_t)(128 * st);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk & 3) * 32;  // 16 columns = 32 bytes inside an atom
+          const uint64_t ad = ptx::smem_desc_sw128(sQ + (kk >> 2) * (kBM * 128) + koff, 16, 1024);
+          const uint64_t bd = ptx::smem_desc_sw128(kb + (kk >> 2) * (BLK * 128) + koff, 16, 1024);
+          ptx::mma_f16_ss(dS, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        ptx::mma_commit(bar(BAR_SFULL + st));
+        ptx::mma_commit(bar(BAR_KEMPTY + ks));
+        return true;
+      };
+      // O_{i%2} += P_i V_i, P_i read from TMEM.
+      auto issue_pv = [&](int i) -> bool {
+        const int vs = i % kVStages;
+        const int st = i & 1;
+        if (!ptx::mbar_wait(bar(BAR_PFULL + st), (i >> 1) & 1, abort_flag, status, kWaitLimitNs,
                             kStatusTimeout))
           return false;
+        if (!ptx::mbar_wait(bar(BAR_VFULL + vs), (i / kVStages) & 1, abort_flag, status,
+                            kWaitLimitNs, kStatusTimeout))
+          return false;
         ptx::tc_fence_after();
-        const uint32_t vs = sV + s * C::kKVBytes;
-        const uint32_t pt = tmem + (uint32_t)(128 * pb);
+        const uint32_t vb = sV + vs * C::kKVBytes;
+        const uint32_t pt = tmem + (uint32_t)(128 * st);
+        const uint32_t dO = tmem + kTmemO + (uint32_t)(128 * st);
 #pragma unroll
         for (int kk = 0; kk < BLK / 16; ++kk) {
           // A = P [128 x BLK] in TMEM: 16 keys = 8 columns of bf16 pairs.
           // B = V [BLK keys x D] read as N x K MN-major: 16 keys = 16 rows of 128 bytes;
           // the D atoms (64 columns each) are BLK*128 bytes apart.
-          const uint64_t bd = ptx::smem_desc_sw128(vs + kk * (16 * 128), BLK * 128, 1024);
-          ptx::mma_f16_ts(tmem + kTmemO, pt + kk * 8, bd, idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+          const uint64_t bd = ptx::smem_desc_sw128(vb + kk * (16 * 128), BLK * 128, 1024);
+          ptx::mma_f16_ts(dO, pt + kk * 8, bd, idesc_o, (i >= 2 || kk > 0) ? 1u : 0u);
         }
-        ptx::mma_commit(bar(BAR_ORDY));
-        ptx::mma_commit(bar(BAR_VEMPTY + s));
-        ptx::mma_commit(bar(BAR_SFREE + pb));
+        ptx::mma_commit(bar(BAR_VEMPTY + vs));
         return true;
       };
+      for (int i = 0; ok && i < n && i < 2; ++i) ok = issue_s(i);
+      // Streams alternate: P_i V_i, then S_{i+2}.  The waits inside suspend the thread
+      // (try_wait), so the MMA warp takes no issue slots from the softmax warps that
+      // share its sub-partition while it waits.
       for (int i = 0; ok && i < n; ++i) {
-        const int s = i & 1;
-        const int sb = i % kSBufs;
-        if (!ptx::mbar_wait(bar(BAR_KFULL + s), (i >> 1) & 1, abort_flag, status, kWaitLimitNs,
-                            kStatusTimeout)) {
-          ok = false;
-          break;
-        }
-        // S/P buffer sb last held P_{i-3}: reusable once P_{i-3} V_{i-3} has completed.
-        if (i >= kSBufs && !ptx::mbar_wait(bar(BAR_SFREE + sb), ((i / kSBufs) - 1) & 1, abort_flag,
-                                           status, kWaitLimitNs, kStatusTimeout)) {
-          ok = false;
-          break;
-        }
-        ptx::tc_fence_after();
-        const uint32_t ks = sK + s * C::kKVBytes;
-        const uint32_t dS = tmem + (uint32_t)(128 * sb);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk & 3) * 32;  // 16 columns = 32 bytes inside an atom
-          const uint64_t ad = ptx::smem_desc_sw128(sQ + (kk >> 2) * (kBM * 128) + koff, 16, 1024);
-          const uint64_t bd = ptx::smem_desc_sw128(ks + (kk >> 2) * (BLK * 128) + koff, 16, 1024);
-          ptx::mma_f16_ss(dS, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
-        }
-        ptx::mma_commit(bar(BAR_SFULL + sb));
-        ptx::mma_commit(bar(BAR_KEMPTY + s));
-        if (i >= 1 && !issue_pv(i - 1)) {
-          ok = false;
-          break;
-        }
+        ok = issue_pv(i);
+        if (ok && i + 2 < n) ok = issue_s(i + 2);
       }
-      if (ok) issue_pv(n - 1);
       // All MMAs this thread issued have completed once BAR_DONE fires.
       ptx::mma_commit(bar(BAR_DONE));
       ptx::mbar_wait(bar(BAR_DONE), 0, nullptr, nullptr, kWaitLimitNs, 0);
-    } else if (warp < 4) {
+    } else if (warp < kSoftmaxWarps) {
       // ------------------------------------------------------------ softmax + epilogue
-      const int r = tid;  // query row == TMEM lane
-      const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+      const int st = warp >> 2;       // stream: kept-list positions st, st+2, st+4, ...
+      const int r = tid & (kBM - 1);  // query row == TMEM lane
+      const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+      const uint32_t srow = tmem + lane_base + (uint32_t)(128 * st);
+      const uint32_t orow_t = tmem + lane_base + kTmemO + (uint32_t)(128 * st);
+      // (dt | dh << 8 | dw << 16) of the columns q*32 + lane this lane evaluates for the
+      // pad-key masks
+      int cpk[BLK / 32];
+#pragma unroll
+      for (int q = 0; q < BLK / 32; ++q) {
+        const int c = q * 32 + lane;
+        const int whw = g.wh * g.ww;
+        const int dt = c / whw;
+        const int dh = (c - dt * whw) / g.ww;
+        const int dw = c - dt * whw - dh * g.ww;
+        cpk[q] = dt | (dh << 8) | (dw << 16);
+      }
+      const int full_ext = g.wt | (g.wh << 8) | (g.ww << 16);
       float m_run = -INFINITY;
       float l_run = 0.f;
       bool ok = true;
-      for (int i = 0; i < n; ++i) {
-        const int sb = i % kSBufs;
-        const int j = list_s[i];
-        const uint32_t srow = tmem + lane_base + (uint32_t)(128 * sb);
+      for (int i = st; i < n; i += 2) {
+        const int t = i >> 1;  // position within the stream
         // Waits are per thread; giving up is decided for the whole warp so that the
         // warp-wide tcgen05 and shuffle operations below stay converged.
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(BAR_SFULL + sb), (i / kSBufs) & 1, abort_flag,
-                                                     status, kWaitLimitNs, kStatusTimeout))) {
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(BAR_SFULL + st), t & 1, abort_flag, status,
+                                                     kWaitLimitNs, kStatusTimeout))) {
           ok = false;
           break;
         }
@@ -288,124 +334,148 @@ __global__ void __launch_bounds__(kThreads, 1)
         float x[BLK];
         {
           // the whole S row in one TMEM load (one round trip)
-          uint32_t t[BLK];
+          uint32_t tt[BLK];
           if constexpr (BLK == 128)
-            ptx::tmem_ld32x128(srow, t);
+            ptx::tmem_ld32x128(srow, tt);
           else
-            ptx::tmem_ld32x64(srow, t);
+            ptx::tmem_ld32x64(srow, tt);
 #pragma unroll
-          for (int c = 0; c < BLK; ++c) x[c] = __uint_as_float(t[c]);
+          for (int c = 0; c < BLK; ++c) x[c] = __uint_as_float(tt[c]);
         }
         // Pad keys of a partial window get -inf; validity is per column, the same for
         // every row, so each lane evaluates 1/32 of the columns and the warp shares bits.
-        int nt, nh, nw;
-        block_extent(g, j, nt, nh, nw);
-        if (nt < g.wt || nh < g.wh || nw < g.ww) {
+        const int ext = ext_s[i];
+        if (ext != full_ext) {
+          const int nt = ext & 255, nh = (ext >> 8) & 255, nw = ext >> 16;
           uint32_t vm[BLK / 32];
-          const int whw = g.wh * g.ww;
 #pragma unroll
-          for (int q = 0; q < BLK / 32; ++q) {
-            const int c = q * 32 + lane;
-            const int dt = c / whw;
-            const int rem = c - dt * whw;
-            const int dh = rem / g.ww;
-            const int dw = rem - dh * g.ww;
-            vm[q] = __ballot_sync(0xffffffffu, dt < nt && dh < nh && dw < nw);
-          }
+          for (int q = 0; q < BLK / 32; ++q)
+            vm[q] = __ballot_sync(0xffffffffu, (cpk[q] & 255) < nt && ((cpk[q] >> 8) & 255) < nh &&
+                                                   (cpk[q] >> 16) < nw);
 #pragma unroll
           for (int c = 0; c < BLK; ++c)
             if (!((vm[c >> 5] >> (c & 31)) & 1u)) x[c] = -INFINITY;
         }
-        // Row max of the raw scores (scale > 0 commutes with max) over 8 independent
-        // chains, so the reduction is not one long dependency chain.
+        // Row max of the raw scores (scale > 0 commutes with max): 8 independent chains
+        // of three-input max instructions.
         float mx8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mx8[e] = x[e];
 #pragma unroll
-        for (int c = 8; c < BLK; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int c = 8; c + 8 < BLK; c += 16)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mx8[e] = ptx::fmax3(mx8[e], x[c + e], x[c + 8 + e]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], x[BLK - 8 + e]);
+        const float mx = ptx::fmax3(ptx::fmax3(mx8[0], mx8[1], mx8[2]), ptx::fmax3(mx8[3], mx8[4], mx8[5]),
+                                    fmaxf(mx8[6], mx8[7]));
         // Running max in exp2 units: only moved when it grows by more than 8, so P <= 2^8
         // and O needs rescaling rarely; the final O / l is unchanged by this.
         const float m_new = fmaxf(m_run, mx * scale_log2);
-        const bool grow = m_new > m_run + 8.0f;  // always true on the first block
+        const bool grow = m_new > m_run + 8.0f;  // always true on the stream's first block
         float alpha = 1.0f;
         if (grow) {
           alpha = ptx::ex2(m_run - m_new);  // 0 on the first block
           l_run *= alpha;
           m_run = m_new;
         }
-        if (i >= 1 && __any_sync(0xffffffffu, grow)) {
-          // O is stable once P_{i-1} V_{i-1} has completed.  S_i completing implies that
-          // P_{i-2} V_{i-2} has (a commit covers every earlier MMA), and P_i V_i cannot
-          // start before this warp publishes P_i, so BAR_ORDY is in phase i-1 or i here
-          // and its parity wait is unambiguous.  tcgen05.ld/st are
-          // warp-wide: the warp rescales its 32 rows of O together, rows that did not
-          // grow with alpha = 1.
-          if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(BAR_ORDY), (i - 1) & 1, abort_flag,
-                                                       status, kWaitLimitNs, kStatusTimeout))) {
-            ok = false;
-            break;
-          }
-          ptx::tc_fence_after();
+        if (t >= 1 && __any_sync(0xffffffffu, grow)) {
+          // This stream's O is stable: its previous P V was issued before S_i, and the
+          // commit that signalled S_i covers every earlier MMA; its next P V needs P_i.
+          // tcgen05.ld/st are warp-wide: the warp rescales its 32 rows together, rows
+          // that did not grow with alpha = 1.
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
-            uint32_t t[32];
-            ptx::tmem_ld32(tmem + lane_base + kTmemO + c * 32, t);
+            uint32_t tt[32];
+            ptx::tmem_ld32(orow_t + c * 32, tt);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) t[e] = __float_as_uint(__uint_as_float(t[e]) * alpha);
-            ptx::tmem_st32(tmem + lane_base + kTmemO + c * 32, t);
+            for (int e = 0; e < 32; ++e) tt[e] = __float_as_uint(__uint_as_float(tt[e]) * alpha);
+            ptx::tmem_st32(orow_t + c * 32, tt);
           }
         }
-        // P = exp2(s * scale_log2 - m_run): one FFMA and one ex2 per element, rounded to
-        // bf16 pairs and written over the first BLK/2 columns of this S buffer (the A
-        // operand of P V); the row sum uses 8 independent accumulators.
+        // P = exp2(s * scale_log2 - m_run), rounded to bf16 pairs and written over the
+        // first BLK/2 columns of this stream's S buffer (the A operand of P V); the row
+        // sum uses four packed partial sums.
         const float neg_m = -m_run;
-        float ls[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ls[e] = 0.f;
+        const uint64_t sc2 = ptx::f2(scale_log2, scale_log2), nm2 = ptx::f2(neg_m, neg_m);
+        uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};  // packed partial row sums
         uint32_t pk[BLK / 2];
 #pragma unroll
         for (int c2 = 0; c2 < BLK / 2; ++c2) {
-          const float p0 = ptx::ex2(fmaf(x[2 * c2], scale_log2, neg_m));
-          const float p1 = ptx::ex2(fmaf(x[2 * c2 + 1], scale_log2, neg_m));
-          ls[(2 * c2) & 7] += p0;
-          ls[(2 * c2 + 1) & 7] += p1;
+          // arguments of a pair in one packed FFMA; one pair in four on the FMA pipe
+          // (the two streams' warps share each sub-partition's exp2 unit)
+          float a0, a1;
+          ptx::f2split(ptx::ffma2(ptx::f2(x[2 * c2], x[2 * c2 + 1]), sc2, nm2), a0, a1);
+          const float p0 = (c2 & 3) == 3 ? ptx::exp2_poly(a0) : ptx::ex2(a0);
+          const float p1 = (c2 & 3) == 3 ? ptx::exp2_poly(a1) : ptx::ex2(a1);
+          ls2[c2 & 3] = ptx::fadd2(ls2[c2 & 3], ptx::f2(p0, p1));
           pk[c2] = ptx::pack_bf16(p0, p1);
         }
-        if constexpr (BLK == 128) {
+        if constexpr (BLK == 128)
           ptx::tmem_st32x64(srow, pk);
-        } else {
+        else
           ptx::tmem_st32(srow, pk);
-        }
         ptx::tmem_wait_st();
-        l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+        {
+          float s0, s1;
+          ptx::f2split(ptx::fadd2(ptx::fadd2(ls2[0], ls2[1]), ptx::fadd2(ls2[2], ls2[3])), s0, s1);
+          l_run += s0 + s1;
+        }
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(BAR_PFULL + sb));
+        if (lane == 0) ptx::mbar_arrive(bar(BAR_PFULL + st));
       }
       // ---------------------------------------------------------- epilogue
-      // BAR_DONE fires once every MMA of the CTA has completed (the softmax skips most
-      // BAR_ORDY phases, so a parity wait there could alias an older phase).
+      // Merge the two streams: m = max(m_0, m_1), f_s = 2^(m_s - m),
+      // O = (f_0 O_0 + f_1 O_1) / (f_0 l_0 + f_1 l_1).  A stream with no block has
+      // l_s = 0 and m_s = -inf (f_s = 0) and its O_s is never read.  Warpgroup s writes
+      // output columns [s*D/2, (s+1)*D/2).
+      float* xch = reinterpret_cast<float*>(smem + C::kOffXch);  // [stream][m, l][128]
+      xch[(st * 2 + 0) * 128 + r] = m_run;
+      xch[(st * 2 + 1) * 128 + r] = l_run;
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(BAR_XCH));
+      ok = ok && __all_sync(0xffffffffu, ptx::mbar_wait(bar(BAR_XCH), 0, abort_flag, status,
+                                                        kWaitLimitNs, kStatusTimeout));
+      // BAR_DONE fires once every MMA of the CTA has completed.
       if (ok && __all_sync(0xffffffffu, ptx::mbar_wait(bar(BAR_DONE), 0, abort_flag, status,
                                                        kWaitLimitNs, kStatusTimeout))) {
         ptx::tc_fence_after();
-        const float inv = l_run > 0.f ? 1.0f / l_run : 0.f;
-        __nv_bfloat16* orow =
-            op + ((brow0 + (long long)qblk * BLK + r) * g.heads + head) * (long long)D;
+        const float m0 = xch[0 * 128 + r], l0 = xch[1 * 128 + r];
+        const float m1 = xch[2 * 128 + r], l1 = xch[3 * 128 + r];
+        const float m = fmaxf(m0, m1);
+        const float f0 = l0 > 0.f ? ptx::ex2(m0 - m) : 0.f;
+        const float f1 = l1 > 0.f ? ptx::ex2(m1 - m) : 0.f;
+        const float den = f0 * l0 + f1 * l1;
+        const float inv = den > 0.f ? 1.0f / den : 0.f;
+        const float w0 = f0 * inv, w1 = f1 * inv;
+        const bool use1 = n > 1;  // stream 1 holds at least one block
+        __nv_bfloat16* orow = op + ((brow0 + (long long)qblk * BLK + r) * g.heads + head) * (long long)D +
+                              st * (D / 2);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t t[32];
-          ptx::tmem_ld32(tmem + lane_base + kTmemO + c * 32, t);
+        for (int c = 0; c < D / 64; ++c) {
+          const uint32_t col = (uint32_t)(st * (D / 2) + c * 32);
+          uint32_t a0[32], a1[32];
+          ptx::tmem_ld32(tmem + lane_base + kTmemO + col, a0);
+          if (use1) {
+            ptx::tmem_ld32(tmem + lane_base + kTmemO + 128 + col, a1);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) a1[e] = 0u;
+          }
           if (r < BLK) {
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
-              uint4 w;
-              w.x = ptx::pack_bf16(__uint_as_float(t[8 * v + 0]) * inv, __uint_as_float(t[8 * v + 1]) * inv);
-              w.y = ptx::pack_bf16(__uint_as_float(t[8 * v + 2]) * inv, __uint_as_float(t[8 * v + 3]) * inv);
-              w.z = ptx::pack_bf16(__uint_as_float(t[8 * v + 4]) * inv, __uint_as_float(t[8 * v + 5]) * inv);
-              w.w = ptx::pack_bf16(__uint_as_float(t[8 * v + 6]) * inv, __uint_as_float(t[8 * v + 7]) * inv);
-              reinterpret_cast<uint4*>(orow + c * 32)[v] = w;
+              float o[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                o[e] = __uint_as_float(a0[8 * v + e]) * w0 + (use1 ? __uint_as_float(a1[8 * v + e]) * w1 : 0.f);
+              uint4 wv;
+              wv.x = ptx::pack_bf16(o[0], o[1]);
+              wv.y = ptx::pack_bf16(o[2], o[3]);
+              wv.z = ptx::pack_bf16(o[4], o[5]);
+              wv.w = ptx::pack_bf16(o[6], o[7]);
+              reinterpret_cast<uint4*>(orow + c * 32)[v] = wv;
             }
           }
         }
@@ -428,6 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 }  // namespace rf2
+
 
 
 namespace rf2 {

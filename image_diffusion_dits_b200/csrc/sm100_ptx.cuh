@@ -49,27 +49,44 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Time-bounded wait for the phase of parity `parity` to complete.  Gives up (returns
-// false) when *abort is set by another thread of the CTA, when the call-wide status word
-// reports an error, or after `limit_ns`; in the last case it raises both flags.
+// Non-blocking test of the phase of parity `parity`.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Time-bounded wait for the phase of parity `parity` to complete.  The poll loop touches
+// nothing but the barrier: every 1024 polls it reads the CTA's abort flag and the clock,
+// and only every 65536 polls the call-wide status word in global memory, so a phase that
+// completes is seen within one poll.  Gives up (returns false) when *abort is set by
+// another thread of the CTA, when the status word reports another CTA's timeout, or after
+// `limit_ns`; in the last case it raises both flags.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           volatile int* gstatus, uint64_t limit_ns,
                                           int timeout_code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
+  uint32_t spins = 0;
   while (true) {
-#pragma unroll 1
-    for (int k = 0; k < 32; ++k)
-      if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if (gstatus != nullptr && *gstatus == timeout_code) {  // another CTA timed out
-      *abort = 1;
-      return false;
-    }
-    if (globaltimer() - t0 > limit_ns) {
-      *abort = 1;
-      if (gstatus != nullptr) atomicCAS((int*)gstatus, 0, timeout_code);
-      return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((++spins & 1023u) == 0u) {
+      if (abort != nullptr && *abort) return false;
+      if (gstatus != nullptr && (spins & 0xFFFFu) == 0u && *gstatus == timeout_code) {
+        *abort = 1;  // another CTA timed out
+        return false;
+      }
+      if (globaltimer() - t0 > limit_ns) {
+        if (abort != nullptr) *abort = 1;
+        if (gstatus != nullptr) atomicCAS((int*)gstatus, 0, timeout_code);
+        return false;
+      }
     }
   }
 }
@@ -209,6 +226,14 @@ __device__ __forceinline__ void tmem_st32x64(uint32_t taddr, const uint32_t (&r)
 }
 
 
+
+// 16 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st32x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -240,6 +265,57 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int b_mn_maj
          | ((uint32_t)b_mn_major << 16)  // B major
          | ((uint32_t)(N >> 3) << 17)    // N / 8
          | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
+// Packed fp32 pairs (sm_100a f32x2 arithmetic): one instruction for two lanes' worth.
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+__device__ __forceinline__ void f2split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// max of three fp32 values in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Named barrier over `count` threads (a multiple of 32), id 1..15.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// 2^x on the FMA pipe, for x <= 64 (the softmax's arguments are <= 8): x = n + f with
+// n = round(x) taken from the low mantissa bits of x + 1.5*2^23 and f in [-0.5, 0.5];
+// 2^f from a cubic fitted here for minimum relative error on [-0.5, 0.5] (max relative
+// error 7.5e-5, far below the bf16 rounding of P); n is added to the exponent field.
+// Arguments below -125 (masked keys, -inf) give 2^-125, which is zero for P in bf16 and
+// negligible in the row sum.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  float p = fmaf(0.05517259240150452f, f, 0.24261370301246643f);
+  p = fmaf(p, f, 0.6932610273361206f);
+  p = fmaf(p, f, 0.9999278783798218f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ float ex2(float x) {
