@@ -238,62 +238,86 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_o = ptx::idesc_bf16_f32(kBM, D, 1);
       bool ok = ptx::mbar_wait(bar(BAR_Q), 0, abort_flag, status, kWaitLimitNs, kStatusTimeout);
       ptx::tc_fence_after();
+      // Shared-memory descriptors of the tile bases; every MMA step only adds a constant
+      // to the start-address field (tiles stay inside the 14-bit address range).
+      const uint64_t qdesc = ptx::smem_desc_sw128(sQ, 16, 1024);
+      const uint64_t kdesc0 = ptx::smem_desc_sw128(sK, 16, 1024);
+      const uint64_t vdesc0 = ptx::smem_desc_sw128(sV, BLK * 128, 1024);
       // S_i into the S/P buffer of stream i%2.  For i >= 2 that buffer holds P_{i-2}, which
       // P_{i-2} V_{i-2} reads; that MMA was issued before this one by this thread, and
       // tcgen05 MMAs issued by one thread execute in issue order, so S_i is issued
       // without waiting for it to complete (no drain of the tensor pipe per block).
-      auto issue_s = [&](int i) -> bool {
+      auto wait_s = [&](int i) -> bool {
+        return ptx::mbar_wait(bar(BAR_KFULL + i % kKStages), (i / kKStages) & 1, abort_flag, status,
+                              kWaitLimitNs, kStatusTimeout);
+      };
+      auto issue_s = [&](int i) {
         const int ks = i % kKStages;
         const int st = i & 1;
-        if (!ptx::mbar_wait(bar(BAR_KFULL + ks), (i / kKStages) & 1, abort_flag, status,
-                            kWaitLimitNs, kStatusTimeout))
-          return false;
-        ptx::tc_fence_after();
-        const uint32_t kb = sK + ks * C::kKVBytes;
+        const uint64_t kdesc = kdesc0 + (uint64_t)((ks * C::kKVBytes) >> 4);
         const uint32_t dS = tmem + (uint32_t)(128 * st);
+        if constexpr (D == 128) {
+          // step kk: atom kk/4, 16 columns = 32 bytes inside it (start address field >> 4)
+          constexpr uint32_t QA = kBM * 128 / 16, KA = BLK * 128 / 16;
+          ptx::mma8_ss<2, 4, 6, QA, QA + 2, QA + 4, QA + 6, 2, 4, 6, KA, KA + 2, KA + 4, KA + 6>(
+              dS, qdesc, kdesc, idesc_s, 0u);
+        } else {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk & 3) * 32;  // 16 columns = 32 bytes inside an atom
-          const uint64_t ad = ptx::smem_desc_sw128(sQ + (kk >> 2) * (kBM * 128) + koff, 16, 1024);
-          const uint64_t bd = ptx::smem_desc_sw128(kb + (kk >> 2) * (BLK * 128) + koff, 16, 1024);
-          ptx::mma_f16_ss(dS, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad = qdesc + (uint64_t)(((kk >> 2) * (kBM * 128) + (kk & 3) * 32) >> 4);
+            const uint64_t bd = kdesc + (uint64_t)(((kk >> 2) * (BLK * 128) + (kk & 3) * 32) >> 4);
+            ptx::mma_f16_ss(dS, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          }
         }
         ptx::mma_commit(bar(BAR_SFULL + st));
         ptx::mma_commit(bar(BAR_KEMPTY + ks));
-        return true;
       };
       // O_{i%2} += P_i V_i, P_i read from TMEM.
-      auto issue_pv = [&](int i) -> bool {
+      auto wait_pv = [&](int i) -> bool {
+        return ptx::mbar_wait(bar(BAR_PFULL + (i & 1)), (i >> 1) & 1, abort_flag, status,
+                              kWaitLimitNs, kStatusTimeout) &&
+               ptx::mbar_wait(bar(BAR_VFULL + i % kVStages), (i / kVStages) & 1, abort_flag, status,
+                              kWaitLimitNs, kStatusTimeout);
+      };
+      auto issue_pv = [&](int i) {
         const int vs = i % kVStages;
         const int st = i & 1;
-        if (!ptx::mbar_wait(bar(BAR_PFULL + st), (i >> 1) & 1, abort_flag, status, kWaitLimitNs,
-                            kStatusTimeout))
-          return false;
-        if (!ptx::mbar_wait(bar(BAR_VFULL + vs), (i / kVStages) & 1, abort_flag, status,
-                            kWaitLimitNs, kStatusTimeout))
-          return false;
-        ptx::tc_fence_after();
-        const uint32_t vb = sV + vs * C::kKVBytes;
+        const uint64_t vdesc = vdesc0 + (uint64_t)((vs * C::kKVBytes) >> 4);
         const uint32_t pt = tmem + (uint32_t)(128 * st);
         const uint32_t dO = tmem + kTmemO + (uint32_t)(128 * st);
-#pragma unroll
-        for (int kk = 0; kk < BLK / 16; ++kk) {
+        if constexpr (BLK == 128) {
           // A = P [128 x BLK] in TMEM: 16 keys = 8 columns of bf16 pairs.
           // B = V [BLK keys x D] read as N x K MN-major: 16 keys = 16 rows of 128 bytes;
           // the D atoms (64 columns each) are BLK*128 bytes apart.
-          const uint64_t bd = ptx::smem_desc_sw128(vb + kk * (16 * 128), BLK * 128, 1024);
-          ptx::mma_f16_ts(dO, pt + kk * 8, bd, idesc_o, (i >= 2 || kk > 0) ? 1u : 0u);
+          ptx::mma8_ts<8, 16, 24, 32, 40, 48, 56, 16 * 128 / 16>(dO, pt, vdesc, idesc_o,
+                                                                  i >= 2 ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < BLK / 16; ++kk) {
+            const uint64_t bd = vdesc + (uint64_t)((kk * (16 * 128)) >> 4);
+            ptx::mma_f16_ts(dO, pt + kk * 8, bd, idesc_o, (i >= 2 || kk > 0) ? 1u : 0u);
+          }
         }
         ptx::mma_commit(bar(BAR_VEMPTY + vs));
-        return true;
       };
-      for (int i = 0; ok && i < n && i < 2; ++i) ok = issue_s(i);
-      // Streams alternate: P_i V_i, then S_{i+2}.  The waits inside suspend the thread
-      // (try_wait), so the MMA warp takes no issue slots from the softmax warps that
-      // share its sub-partition while it waits.
+      for (int i = 0; ok && i < n && i < 2; ++i) {
+        ok = wait_s(i);
+        if (ok) {
+          ptx::tc_fence_after();
+          issue_s(i);
+        }
+      }
+      // Streams alternate: P_i V_i, then S_{i+2}.  All three inputs are awaited before
+      // either group is issued, so the two groups go to the tensor pipe back to back.
+      // The waits suspend the thread (try_wait), so the MMA warp takes no issue slots
+      // from the softmax warps that share its sub-partition while it waits.  (Two
+      // issuing threads, one per stream, measured slower: the interleaved chains.)
       for (int i = 0; ok && i < n; ++i) {
-        ok = issue_pv(i);
-        if (ok && i + 2 < n) ok = issue_s(i + 2);
+        ok = wait_pv(i) && (i + 2 >= n || wait_s(i + 2));
+        if (!ok) break;
+        ptx::tc_fence_after();
+        issue_pv(i);
+        if (i + 2 < n) issue_s(i + 2);
       }
       // All MMAs this thread issued have completed once BAR_DONE fires.
       ptx::mma_commit(bar(BAR_DONE));

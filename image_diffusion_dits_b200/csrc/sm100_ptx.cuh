@@ -71,6 +71,7 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           volatile int* gstatus, uint64_t limit_ns,
                                           int timeout_code) {
+  if (mbar_test_wait(bar, parity)) return true;  // already complete: no suspend logic
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   uint32_t spins = 0;
@@ -154,6 +155,70 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+
+// Eight consecutive K=16 steps of one MMA chain in a single asm block: step k uses the
+// descriptors (a0 + k*A_STEP_k, b0 + k*B_STEP_k) where the per-step increments (in the
+// descriptors' 16-byte address units) are compile-time constants passed as immediates.
+// Step 0 accumulates when `acc0` != 0, later steps always accumulate.  A in shared memory.
+template <uint32_t A1, uint32_t A2, uint32_t A3, uint32_t A4, uint32_t A5, uint32_t A6, uint32_t A7,
+          uint32_t B1, uint32_t B2, uint32_t B3, uint32_t B4, uint32_t B5, uint32_t B6, uint32_t B7>
+__device__ __forceinline__ void mma8_ss(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc,
+                                        uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred p0, p1;\n\t.reg .b64 a, b;\n\t"
+      "setp.ne.b32 p0, %4, 0;\n\t"
+      "setp.eq.b32 p1, %4, %4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p0;\n\t"
+      "add.s64 a, %1, %5;\n\tadd.s64 b, %2, %12;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, p1;\n\t"
+      "add.s64 a, %1, %6;\n\tadd.s64 b, %2, %13;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, p1;\n\t"
+      "add.s64 a, %1, %7;\n\tadd.s64 b, %2, %14;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, p1;\n\t"
+      "add.s64 a, %1, %8;\n\tadd.s64 b, %2, %15;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, p1;\n\t"
+      "add.s64 a, %1, %9;\n\tadd.s64 b, %2, %16;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, p1;\n\t"
+      "add.s64 a, %1, %10;\n\tadd.s64 b, %2, %17;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, p1;\n\t"
+      "add.s64 a, %1, %11;\n\tadd.s64 b, %2, %18;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, p1;\n\t}" ::"r"(d_tmem),
+      "l"(a0), "l"(b0), "r"(idesc), "r"(acc0), "n"(A1), "n"(A2), "n"(A3), "n"(A4), "n"(A5),
+      "n"(A6), "n"(A7), "n"(B1), "n"(B2), "n"(B3), "n"(B4), "n"(B5), "n"(B6), "n"(B7)
+      : "memory");
+}
+
+// Same with A in TMEM: step k reads A at column a0 + 8k (16 bf16 K-elements = 8 columns
+// of pairs) unless an explicit column offset table is given, B descriptor b0 + k*B_STEP.
+template <uint32_t AC1, uint32_t AC2, uint32_t AC3, uint32_t AC4, uint32_t AC5, uint32_t AC6,
+          uint32_t AC7, uint32_t BS>
+__device__ __forceinline__ void mma8_ts(uint32_t d_tmem, uint32_t a0, uint64_t b0, uint32_t idesc,
+                                        uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred p0, p1;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
+      "setp.ne.b32 p0, %4, 0;\n\t"
+      "setp.eq.b32 p1, %4, %4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n\t"
+      "add.s32 a, %1, %5;\n\tadd.s64 b, %2, %12;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, p1;\n\t"
+      "add.s32 a, %1, %6;\n\tadd.s64 b, %2, %13;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, p1;\n\t"
+      "add.s32 a, %1, %7;\n\tadd.s64 b, %2, %14;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, p1;\n\t"
+      "add.s32 a, %1, %8;\n\tadd.s64 b, %2, %15;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, p1;\n\t"
+      "add.s32 a, %1, %9;\n\tadd.s64 b, %2, %16;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, p1;\n\t"
+      "add.s32 a, %1, %10;\n\tadd.s64 b, %2, %17;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, p1;\n\t"
+      "add.s32 a, %1, %11;\n\tadd.s64 b, %2, %18;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, p1;\n\t}" ::"r"(d_tmem),
+      "r"(a0), "l"(b0), "r"(idesc), "r"(acc0), "n"(AC1), "n"(AC2), "n"(AC3), "n"(AC4), "n"(AC5),
+      "n"(AC6), "n"(AC7), "n"(1 * BS), "n"(2 * BS), "n"(3 * BS), "n"(4 * BS), "n"(5 * BS),
+      "n"(6 * BS), "n"(7 * BS)
       : "memory");
 }
 
