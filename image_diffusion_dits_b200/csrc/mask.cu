@@ -73,67 +73,71 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const int4* __restri
 
 // ------------------------------------------------------------------------------- scores
 // CTA computes a 64 x 64 tile of s = qbar kbar^T * scale for one (b, head); 256 threads,
-// each a 4 x 4 register tile.  D is consumed in slabs of 32 through shared memory,
-// stored d-major so that a thread's 4 rows (and 4 columns) are one float4.
+// each a 4 x 4 register tile.  Both 64 x D operand tiles are staged in shared memory in
+// one pass (one exposed L2 latency per CTA), stored d-major with rows padded to 68
+// floats so that a thread's 4 rows (and 4 columns) are one aligned float4 and the
+// transposing stores hit distinct banks.  Every score is a sequential fmaf chain over d.
 constexpr int kSTile = 64;
-constexpr int kSSlab = 32;
+constexpr int kSPad = kSTile + 4;
 
+template <int D>
 __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ qbar,
                                                      const float* __restrict__ kbar,
                                                      float* __restrict__ s, Geo g, float scale) {
-  __shared__ __align__(16) float qs[kSSlab][kSTile];
-  __shared__ __align__(16) float ks[kSSlab][kSTile];
+  extern __shared__ __align__(16) float ssm[];
+  float* qs = ssm;               // [D][kSPad]
+  float* ks = ssm + D * kSPad;   // [D][kSPad]
   const int bh = blockIdx.z;
   const int i0 = blockIdx.y * kSTile;
   const int j0 = blockIdx.x * kSTile;
-  const float* qb = qbar + (long long)bh * g.Nb * g.D;
-  const float* kb = kbar + (long long)bh * g.Nb * g.D;
+  const float* qb = qbar + (long long)bh * g.Nb * D;
+  const float* kb = kbar + (long long)bh * g.Nb * D;
   const int tid = threadIdx.x;
   const int ti = tid >> 4;   // rows 4*ti .. 4*ti+3
   const int tj = tid & 15;   // cols 4*tj .. 4*tj+3
+  // fill: consecutive threads take consecutive rows of the same 4 d
+#pragma unroll 4
+  for (int f = tid; f < kSTile * D / 4; f += 256) {
+    const int r = f % kSTile, d4 = f / kSTile;
+    const int gi = i0 + r, gj = j0 + r;
+    const float4 qv = gi < g.Nb ? __ldg(reinterpret_cast<const float4*>(qb + (long long)gi * D) + d4)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 kv = gj < g.Nb ? __ldg(reinterpret_cast<const float4*>(kb + (long long)gj * D) + d4)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+    qs[(4 * d4 + 0) * kSPad + r] = qv.x;
+    qs[(4 * d4 + 1) * kSPad + r] = qv.y;
+    qs[(4 * d4 + 2) * kSPad + r] = qv.z;
+    qs[(4 * d4 + 3) * kSPad + r] = qv.w;
+    ks[(4 * d4 + 0) * kSPad + r] = kv.x;
+    ks[(4 * d4 + 1) * kSPad + r] = kv.y;
+    ks[(4 * d4 + 2) * kSPad + r] = kv.z;
+    ks[(4 * d4 + 3) * kSPad + r] = kv.w;
+  }
+  __syncthreads();
   float acc[4][4];
 #pragma unroll
   for (int a = 0; a < 4; ++a)
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
-  for (int d0 = 0; d0 < g.D; d0 += kSSlab) {
-    // Slab fill: 64 rows x 32 d of each operand as 512 float4 per operand.  Within a
-    // warp consecutive threads take consecutive rows of the same 4 d, so the transposed
-    // (d-major) shared-memory stores hit 32 different banks.
-#pragma unroll
-    for (int it = 0; it < (kSTile * kSSlab / 4) / 256; ++it) {
-      const int f = tid + 256 * it;
-      const int r = f % kSTile, d4 = f / kSTile;
-      const int gi = i0 + r, gj = j0 + r;
-      float4 qv = gi < g.Nb ? *reinterpret_cast<const float4*>(qb + (long long)gi * g.D + d0 + 4 * d4)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-      float4 kv = gj < g.Nb ? *reinterpret_cast<const float4*>(kb + (long long)gj * g.D + d0 + 4 * d4)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-      qs[4 * d4 + 0][r] = qv.x; qs[4 * d4 + 1][r] = qv.y; qs[4 * d4 + 2][r] = qv.z; qs[4 * d4 + 3][r] = qv.w;
-      ks[4 * d4 + 0][r] = kv.x; ks[4 * d4 + 1][r] = kv.y; ks[4 * d4 + 2][r] = kv.z; ks[4 * d4 + 3][r] = kv.w;
-    }
-    __syncthreads();
 #pragma unroll 8
-    for (int d = 0; d < kSSlab; ++d) {
-      float4 qv = reinterpret_cast<const float4*>(qs[d])[ti];
-      float4 kv = reinterpret_cast<const float4*>(ks[d])[tj];
-      float qa[4] = {qv.x, qv.y, qv.z, qv.w};
-      float ka[4] = {kv.x, kv.y, kv.z, kv.w};
+  for (int d = 0; d < D; ++d) {
+    const float4 qv = reinterpret_cast<const float4*>(qs + d * kSPad)[ti];
+    const float4 kv = reinterpret_cast<const float4*>(ks + d * kSPad)[tj];
+    const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
+    const float ka[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[a][c] = fmaf(qa[a], ka[c], acc[a][c]);
-    }
-    __syncthreads();
+      for (int c = 0; c < 4; ++c) acc[a][c] = fmaf(qa[a], ka[c], acc[a][c]);
   }
   float* sb = s + (long long)bh * g.Nb * g.Nb;
 #pragma unroll
   for (int a = 0; a < 4; ++a) {
-    int gi = i0 + 4 * ti + a;
+    const int gi = i0 + 4 * ti + a;
     if (gi >= g.Nb) continue;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      int gj = j0 + 4 * tj + c;
+      const int gj = j0 + 4 * tj + c;
       if (gj < g.Nb) sb[(long long)gi * g.Nb + gj] = acc[a][c] * scale;
     }
   }
@@ -236,11 +240,27 @@ cudaError_t launch_pool(const void* qp, const void* kp, float* qbar, float* kbar
   return cudaGetLastError();
 }
 
+template <int D>
+cudaError_t launch_scores_d(const float* qbar, const float* kbar, float* scores, const Geo& g,
+                            float scale, cudaStream_t s) {
+  const int smem = 2 * D * kSPad * (int)sizeof(float);
+  static int configured_device = -1;  // one flag per instance (per D)
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t e = cudaFuncSetAttribute(scores_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  dim3 grid((g.Nb + kSTile - 1) / kSTile, (g.Nb + kSTile - 1) / kSTile, g.B * g.heads);
+  scores_kernel<D><<<grid, 256, smem, s>>>(qbar, kbar, scores, g, scale);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_scores(const float* qbar, const float* kbar, float* scores, const Geo& g,
                           float scale, cudaStream_t s) {
-  dim3 grid((g.Nb + kSTile - 1) / kSTile, (g.Nb + kSTile - 1) / kSTile, g.B * g.heads);
-  scores_kernel<<<grid, 256, 0, s>>>(qbar, kbar, scores, g, scale);
-  return cudaGetLastError();
+  if (g.D == 128) return launch_scores_d<128>(qbar, kbar, scores, g, scale, s);
+  return launch_scores_d<64>(qbar, kbar, scores, g, scale, s);
 }
 
 cudaError_t launch_topk(const float* scores, int32_t* idx, int32_t* cnt, int kmax, int kept,
