@@ -136,6 +136,24 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(rows)}
 
 
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank timings (the job's time is its slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def job_throughput(flop_per_call, world, ms_per_call):
+    """Whole-job dense-equivalent TFLOP/s: every rank runs one call per step, so the job
+    processes world * flop_per_call per (max over ranks) step time."""
+    return flop_per_call * world / (ms_per_call * 1e-3) / 1e12
+
+
 def run_cpu_baseline(wl, sparsity, seconds, rows_cap=64):
     """The fp64 oracle on a bounded sample of the same call: its mask stage on the full
     call is skipped (attention dominates); attention is timed on sampled (head, query
@@ -291,12 +309,10 @@ def main():
     total_ms = start.elapsed_time(end)
     seg_ms = [sum(seg_ev[s][i].elapsed_time(seg_ev[s][i + 1]) for s in range(a.steps)) / a.steps
               for i in range(n_seg)]
-    if world > 1:
-        t = torch.tensor([total_ms] + seg_ms, dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms, seg_ms = float(t[0]), [float(x) for x in t[1:]]
+    reduced = max_over_ranks([total_ms] + seg_ms, dev)
+    total_ms, seg_ms = reduced[0], reduced[1:]
     ms_per_step = total_ms / a.steps
-    value = dense * world / (ms_per_step * 1e-3) / 1e12
+    value = job_throughput(dense, world, ms_per_step)
     peaks = _peaks()
 
     # end to end through the public fused call: pinned host inputs in, host output back
@@ -321,12 +337,8 @@ def main():
             ho.copy_(o, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = e0.elapsed_time(e1) / a.steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t[0])
-        e2e = {"value": dense * world / (e2e_ms * 1e-3) / 1e12, "unit": unit, "ms_per_call": e2e_ms,
+        e2e_ms = max_over_ranks([e0.elapsed_time(e1) / a.steps], dev)[0]
+        e2e = {"value": job_throughput(dense, world, e2e_ms), "unit": unit, "ms_per_call": e2e_ms,
                "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": o.numel() * 2}
         del ws, dq, dk, dv
 
