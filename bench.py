@@ -62,7 +62,8 @@ def _peaks():
 def _geometry_numbers(g, kept):
     dense = 4.0 * g.B * g.heads * float(g.N) ** 2 * g.D
     kept_flop = 4.0 * g.B * g.heads * g.Nb * kept * g.blk * g.blk * g.D
-    mask_bytes = 2.0 * g.B * g.Npad * g.heads * g.D * 2  # padded Q and K read once
+    # real (unpadded) rows of Q and K read once, kept lists and counts written once
+    mask_bytes = 2.0 * g.B * g.N * g.heads * g.D * 2 + 4.0 * g.B * g.heads * g.Nb * (kept + 1)
     permute_bytes = 3.0 * g.B * (g.N + g.Npad) * g.heads * g.D * 2
     unpermute_bytes = 1.0 * g.B * (g.N + g.Npad) * g.heads * g.D * 2
     return dense, kept_flop, mask_bytes, permute_bytes, unpermute_bytes

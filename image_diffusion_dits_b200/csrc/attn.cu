@@ -526,14 +526,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 
 namespace rf2 {
-namespace {
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
+EncodeTiledFn tensor_map_encoder() {
   static EncodeTiledFn fn = nullptr;
   if (fn == nullptr) {
     void* p = nullptr;
@@ -546,10 +540,12 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+namespace {
+
 // 3-D view of a [B*Npad, heads, D] bf16 tensor; box = 64 columns x 1 head x `rows` tokens,
 // 128-byte swizzle (one 128-byte row per token, 8-row swizzle atoms of 1024 bytes).
 bool make_map(CUtensorMap* m, const void* base, const Geo& g, int rows) {
-  EncodeTiledFn fn = encode_fn();
+  EncodeTiledFn fn = tensor_map_encoder();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {(cuuint64_t)g.D, (cuuint64_t)g.heads, (cuuint64_t)(g.B * g.Npad)};
   cuuint64_t strides[2] = {(cuuint64_t)g.D * 2, (cuuint64_t)g.heads * g.D * 2};

@@ -4,10 +4,13 @@
 //
 //   pool   : qbar/kbar[b, head, j, :] = fp32 mean of the real tokens of block j.
 //            HBM-bound streaming reduction over the permuted Q and K.
-//   scores : s[b, head, i, j] = qbar_i . kbar_j * scale, an fp32 register-tiled product.
+//   scores : s[b, head, i, j] = qbar_i . kbar_j * scale on the tensor cores: each mean is
+//            split into three bf16 parts (hi + mid + lo, about 24 significant bits) and
+//            the six products that matter at fp32 precision are accumulated in fp32.
 //   topk   : per row, the sink blocks plus the m best other blocks (ties to the lower
 //            id) as an ascending list; one warp per row, exact bitwise search.
 #include "rf2_common.cuh"
+#include "sm100_ptx.cuh"
 
 namespace rf2 {
 namespace {
@@ -31,8 +34,8 @@ __device__ __forceinline__ void acc_bf16x8(float (&a)[8], const int4& v) {
 
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const int4* __restrict__ qp,
                                                             const int4* __restrict__ kp,
-                                                            float* __restrict__ qbar,
-                                                            float* __restrict__ kbar, Geo g,
+                                                            __nv_bfloat16* __restrict__ q3,
+                                                            __nv_bfloat16* __restrict__ k3, Geo g,
                                                             int chunks) {
   const int c = blockIdx.x * kPoolThreads + threadIdx.x;
   const int j = blockIdx.y;
@@ -64,90 +67,175 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const int4* __restri
   const int ch = c * 8;           // channel within heads*D
   const int head = ch / g.D;
   const int d = ch - head * g.D;
-  float* dst = (which ? kbar : qbar) + (((long long)b * g.heads + head) * g.Nb + j) * g.D + d;
-  float4 o0 = make_float4(a[0] * inv, a[1] * inv, a[2] * inv, a[3] * inv);
-  float4 o1 = make_float4(a[4] * inv, a[5] * inv, a[6] * inv, a[7] * inv);
-  reinterpret_cast<float4*>(dst)[0] = o0;
-  reinterpret_cast<float4*>(dst)[1] = o1;
+  // the mean x in three bf16 parts: hi = bf16(x), mid = bf16(x - hi), lo = bf16(x - hi - mid);
+  // both differences are exact in fp32
+  const long long R = (long long)g.B * g.heads * g.Nb;
+  __nv_bfloat16* dst = (which ? k3 : q3) + (((long long)b * g.heads + head) * g.Nb + j) * g.D + d;
+  uint32_t part[3][4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    float x2[2] = {a[2 * e] * inv, a[2 * e + 1] * inv};
+    uint16_t hb[3][2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float r = x2[h];
+#pragma unroll
+      for (int q = 0; q < 3; ++q) {
+        const __nv_bfloat16 v = __float2bfloat16_rn(r);
+        hb[q][h] = __bfloat16_as_ushort(v);
+        r -= __bfloat162float(v);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 3; ++q) part[q][e] = (uint32_t)hb[q][0] | ((uint32_t)hb[q][1] << 16);
+  }
+#pragma unroll
+  for (int q = 0; q < 3; ++q)
+    *reinterpret_cast<uint4*>(dst + q * R * g.D) = make_uint4(part[q][0], part[q][1], part[q][2], part[q][3]);
 }
 
 // ------------------------------------------------------------------------------- scores
-// CTA computes a 64 x 64 tile of s = qbar kbar^T * scale for one (b, head); 256 threads,
-// each a 4 x 4 register tile.  Both 64 x D operand tiles are staged in shared memory in
-// one pass (one exposed L2 latency per CTA), stored d-major with rows padded to 68
-// floats so that a thread's 4 rows (and 4 columns) are one aligned float4 and the
-// transposing stores hit distinct banks.  Every score is a sequential fmaf chain over d.
-constexpr int kSTile = 64;
-constexpr int kSPad = kSTile + 4;
+// One CTA per 128 x 128 tile of s for one (b, head).  D is taken 64 columns at a time:
+// the three bf16 parts of 128 query means (A) and 128 key means (B) for those columns
+// (48 KB) are loaded by TMA (128-byte swizzle, the same K-major layout as the attention
+// kernel's Q and K tiles) and thread 0 issues, into one fp32 TMEM accumulator, the
+// products lo.hi, hi.lo, mid.mid, mid.hi, hi.mid, hi.hi (smallest first); the dropped
+// products are below 2^-24 of the score.  With 48 KB of staging, several CTAs share an
+// SM and one's loads overlap another's products and stores.  The four warps then read
+// their 32 rows from TMEM and store s * scale.  Rows or columns past Nb in a tile come
+// from the next head's means (or TMA zero fill) and are not stored.
+constexpr int kSTile = 128;
+constexpr int kSThreads = 128;
+constexpr uint64_t kScoresWaitNs = 500ull * 1000ull * 1000ull;
 
 template <int D>
-__global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ qbar,
-                                                     const float* __restrict__ kbar,
-                                                     float* __restrict__ s, Geo g, float scale) {
-  extern __shared__ __align__(16) float ssm[];
-  float* qs = ssm;               // [D][kSPad]
-  float* ks = ssm + D * kSPad;   // [D][kSPad]
-  const int bh = blockIdx.z;
-  const int i0 = blockIdx.y * kSTile;
-  const int j0 = blockIdx.x * kSTile;
-  const float* qb = qbar + (long long)bh * g.Nb * D;
-  const float* kb = kbar + (long long)bh * g.Nb * D;
-  const int tid = threadIdx.x;
-  const int ti = tid >> 4;   // rows 4*ti .. 4*ti+3
-  const int tj = tid & 15;   // cols 4*tj .. 4*tj+3
-  // fill: consecutive threads take consecutive rows of the same 4 d
-#pragma unroll 4
-  for (int f = tid; f < kSTile * D / 4; f += 256) {
-    const int r = f % kSTile, d4 = f / kSTile;
-    const int gi = i0 + r, gj = j0 + r;
-    const float4 qv = gi < g.Nb ? __ldg(reinterpret_cast<const float4*>(qb + (long long)gi * D) + d4)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4 kv = gj < g.Nb ? __ldg(reinterpret_cast<const float4*>(kb + (long long)gj * D) + d4)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-    qs[(4 * d4 + 0) * kSPad + r] = qv.x;
-    qs[(4 * d4 + 1) * kSPad + r] = qv.y;
-    qs[(4 * d4 + 2) * kSPad + r] = qv.z;
-    qs[(4 * d4 + 3) * kSPad + r] = qv.w;
-    ks[(4 * d4 + 0) * kSPad + r] = kv.x;
-    ks[(4 * d4 + 1) * kSPad + r] = kv.y;
-    ks[(4 * d4 + 2) * kSPad + r] = kv.z;
-    ks[(4 * d4 + 3) * kSPad + r] = kv.w;
+struct ScoresCfg {
+  static constexpr int kChunks = D / 64;                         // 64-column slices of D
+  static constexpr int kPartBytes = kSTile * 64 * 2;             // one part of one operand, one slice
+  static constexpr int kOffA = 0;                                // 3 parts of A
+  static constexpr int kOffB = 3 * kPartBytes;                   // 3 parts of B
+  static constexpr int kOffBar = 6 * kPartBytes;                 // full + done barriers
+  static constexpr int kSmem = kOffBar + 64 + 1024;              // + alignment slack
+};
+
+template <int D>
+__global__ void __launch_bounds__(kSThreads) scores_kernel(const __grid_constant__ CUtensorMap ta,
+                                                              const __grid_constant__ CUtensorMap tb,
+                                                              float* __restrict__ s, Geo g, float scale,
+                                                              int* __restrict__ status) {
+  using C = ScoresCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_s;
+  const uint32_t sbase = ptx::smem_u32(smem);
+  const uint32_t bar_full = sbase + C::kOffBar, bar_free = bar_full + 8, bar_done = bar_full + 16;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long bh = blockIdx.z;
+  const int i0 = blockIdx.y * kSTile, j0 = blockIdx.x * kSTile;
+  const long long R = (long long)g.B * g.heads * g.Nb;  // rows of one part
+  if (warp == 0) {
+    ptx::tmem_alloc(ptx::smem_u32(&tmem_slot), kSTile);
+    ptx::tmem_relinquish();
   }
+  if (threadIdx.x == 32) {
+    ptx::mbar_init(bar_full, 1);
+    ptx::mbar_init(bar_free, 1);
+    ptx::mbar_init(bar_done, 1);
+    abort_s = 0;
+    ptx::fence_mbar_init();
+  }
+  ptx::tc_fence_before();
   __syncthreads();
-  float acc[4][4];
+  ptx::tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  volatile int* abort_flag = &abort_s;
+  if (threadIdx.x == 0) {
+    ptx::prefetch_tmap(&ta);
+    ptx::prefetch_tmap(&tb);
+    constexpr uint32_t idesc = ptx::idesc_bf16_f32(kSTile, kSTile, 0);
+    constexpr int kPairs[6][2] = {{2, 0}, {0, 2}, {1, 1}, {1, 0}, {0, 1}, {0, 0}};  // (A part, B part)
+    bool ok = true;
+    int issued = 0;  // slices whose loads were issued
+    for (int kc = 0; ok && kc < C::kChunks; ++kc) {
+      // the staging buffers are free once the previous slice's products completed
+      if (kc > 0) ok = ptx::mbar_wait(bar_free, (kc - 1) & 1, abort_flag, status, kScoresWaitNs, kStatusTimeout);
+      if (!ok) break;
+      ptx::mbar_arrive_expect_tx(bar_full, 6 * C::kPartBytes);
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+      for (int q = 0; q < 3; ++q) {
+        ptx::tma_load_2d(sbase + C::kOffA + q * C::kPartBytes, &ta, bar_full, kc * 64,
+                         (int)(q * R + bh * g.Nb + i0));
+        ptx::tma_load_2d(sbase + C::kOffB + q * C::kPartBytes, &tb, bar_full, kc * 64,
+                         (int)(q * R + bh * g.Nb + j0));
+      }
+      issued = kc + 1;
+      ok = ptx::mbar_wait(bar_full, kc & 1, abort_flag, status, kScoresWaitNs, kStatusTimeout);
+      if (!ok) break;
+      ptx::tc_fence_after();
 #pragma unroll
-    for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
-#pragma unroll 8
-  for (int d = 0; d < D; ++d) {
-    const float4 qv = reinterpret_cast<const float4*>(qs + d * kSPad)[ti];
-    const float4 kv = reinterpret_cast<const float4*>(ks + d * kSPad)[tj];
-    const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
-    const float ka[4] = {kv.x, kv.y, kv.z, kv.w};
+      for (int pr = 0; pr < 6; ++pr) {
+        const uint64_t ad = ptx::smem_desc_sw128(sbase + C::kOffA + kPairs[pr][0] * C::kPartBytes, 16, 1024);
+        const uint64_t bd = ptx::smem_desc_sw128(sbase + C::kOffB + kPairs[pr][1] * C::kPartBytes, 16, 1024);
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[a][c] = fmaf(qa[a], ka[c], acc[a][c]);
-  }
-  float* sb = s + (long long)bh * g.Nb * g.Nb;
-#pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int gi = i0 + 4 * ti + a;
-    if (gi >= g.Nb) continue;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int gj = j0 + 4 * tj + c;
-      if (gj < g.Nb) sb[(long long)gi * g.Nb + gj] = acc[a][c] * scale;
+        for (int kk = 0; kk < 4; ++kk)  // 16 columns = 32 bytes of the swizzled 128-byte rows
+          ptx::mma_f16_ss(tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc,
+                          (kc > 0 || pr > 0 || kk > 0) ? 1u : 0u);
+      }
+      ptx::mma_commit(bar_free);
     }
+    if (!ok && issued > 0)  // let the copies in flight land before the CTA exits
+      ptx::mbar_wait(bar_full, (issued - 1) & 1, nullptr, nullptr, kScoresWaitNs, 0);
+    // Arrives once every MMA issued above has completed (at once if none was issued);
+    // this thread waits for it without the abort flag, so that no MMA is in flight when
+    // the tensor memory is released.
+    ptx::mma_commit(bar_done);
+    ptx::mbar_wait(bar_done, 0, nullptr, nullptr, kScoresWaitNs, 0);
+  }
+  __syncwarp();
+  const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_done, 0, abort_flag, status, kScoresWaitNs,
+                                                         kStatusTimeout)) &&
+                  *abort_flag == 0;
+  if (ok) {
+    ptx::tc_fence_after();
+    const int r = warp * 32 + lane;  // tile row == TMEM lane
+    const int gi = i0 + r;
+    float* srow = s + (bh * g.Nb + gi) * (long long)g.Nb + j0;
+    const bool vec = (g.Nb & 3) == 0;
+#pragma unroll 1
+    for (int c = 0; c < kSTile / 32; ++c) {
+      uint32_t v[32];
+      ptx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c * 32, v);
+      if (gi < g.Nb) {
+        const int cb = c * 32;
+        if (vec && j0 + cb + 32 <= g.Nb) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            reinterpret_cast<float4*>(srow + cb)[e] =
+                make_float4(__uint_as_float(v[4 * e]) * scale, __uint_as_float(v[4 * e + 1]) * scale,
+                            __uint_as_float(v[4 * e + 2]) * scale, __uint_as_float(v[4 * e + 3]) * scale);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (j0 + cb + e < g.Nb) srow[cb + e] = __uint_as_float(v[e]) * scale;
+        }
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kSTile);
   }
 }
 
 // ------------------------------------------------------------------------------- top-k
 // One warp per (b, head, i) row.  Scores map to order-preserving uint32 keys (every real
-// key is > 0; 0 marks a non-candidate).  The m-th largest candidate key is found exactly
-// by a 32-step bitwise search with warp-wide counts; candidates above it are kept, and
-// equal ones in ascending block order until m are kept.  The output list (sink blocks and kept candidates) is
+// key is > 0; 0 marks a non-candidate).  The threshold is found exactly by a bracketed
+// search over the key range with warp-wide counts (interpolated and bisection steps in
+// turn), stopping as soon as exactly m candidates lie at or above it; candidates above it
+// are kept, and equal ones in ascending block order until m are kept.  The output list (sink blocks and kept candidates) is
 // emitted in ascending order with ballots.
 constexpr int kTopkWarps = 8;
 constexpr int kMaxPerLane = 32;  // Nb <= 1024
@@ -158,59 +246,120 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 }
 
 template <int KPL>
+__device__ __forceinline__ int count_ge(const uint32_t (&key)[KPL], uint32_t t) {
+  int c = 0;
+#pragma unroll
+  for (int k = 0; k < KPL; ++k) c += key[k] >= t;
+  return (int)__reduce_add_sync(0xffffffffu, (uint32_t)c);
+}
+
+template <int KPL>
 __device__ __forceinline__ void topk_row(const float* __restrict__ sr, int32_t* __restrict__ out,
                                          int32_t* __restrict__ cnt_out, int Nb, int kmax, int kept,
                                          int nsink, int lane) {
   uint32_t key[KPL];
+  uint32_t kmin = 0xffffffffu, kmax_key = 0u;
 #pragma unroll
   for (int k = 0; k < KPL; ++k) {
     const int j = k * 32 + lane;
     key[k] = (j < Nb && j >= nsink) ? order_key(__ldg(sr + j)) : 0u;
+    if (key[k] != 0u) kmin = min(kmin, key[k]);
+    kmax_key = max(kmax_key, key[k]);
   }
   const int m = kept - nsink;
   const int ncand = Nb - nsink;
-  uint32_t thr = 0;   // the m-th largest candidate key
-  int take_eq = 0;    // how many keys equal to thr are kept (lowest ids first)
-  if (m > 0 && m < ncand) {
-    // Bitwise search from the most significant bit: the largest t with
-    // #{key >= t} >= m is the m-th largest key.
-#pragma unroll 1
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t t = thr | (1u << bit);
-      int c = 0;
-#pragma unroll
-      for (int k = 0; k < KPL; ++k) c += key[k] >= t;
-      if ((int)__reduce_add_sync(0xffffffffu, (uint32_t)c) >= m) thr = t;
-    }
-    int above = 0;
-#pragma unroll
-    for (int k = 0; k < KPL; ++k) above += key[k] > thr;
-    take_eq = m - (int)__reduce_add_sync(0xffffffffu, (uint32_t)above);
+  uint32_t thr;       // every candidate key >= thr is kept when take_eq covers all keys == thr
+  if (m <= 0) {
+    thr = 0xffffffffu;  // none (no real key reaches the top value: keys are < 2^32 - 1 or
+                        // equal to it only for NaN patterns, which the ordering puts last)
   } else if (m >= ncand) {
-    thr = 1u;  // every candidate
+    thr = 1u;           // every candidate
   } else {
-    thr = 0xffffffffu;  // m == 0: none
+    // Bracket [lo, hi): #{key >= lo} = c_lo >= m > c_hi = #{key >= hi}.  Each step tries a
+    // t inside the bracket, interpolated from the two counts (keys of a smooth score
+    // distribution are close to uniform locally) on even steps and the midpoint on odd
+    // steps, and stops when exactly m keys are >= t.  Otherwise the bracket shrinks to
+    // one value: lo is then the m-th largest key.
+    uint64_t lo = __reduce_min_sync(0xffffffffu, kmin);
+    uint64_t hi = (uint64_t)__reduce_max_sync(0xffffffffu, kmax_key) + 1u;
+    int c_lo = ncand, c_hi = 0;
+    bool exact = false;
+#pragma unroll 1
+    for (int step = 0; hi - lo > 1; ++step) {
+      const uint64_t w = hi - lo;
+      uint64_t off;
+      if (step & 1) {
+        off = w >> 1;
+      } else {
+        const float frac = (float)(c_lo - m) / (float)(c_lo - c_hi);
+        off = (uint64_t)((double)w * (double)frac);
+      }
+      off = off < 1 ? 1 : (off > w - 1 ? w - 1 : off);
+      const uint32_t t = (uint32_t)(lo + off);
+      const int c = count_ge<KPL>(key, t);
+      if (c == m) {
+        lo = t;
+        exact = true;
+        break;
+      }
+      if (c > m) {
+        lo = t;
+        c_lo = c;
+      } else {
+        hi = t;
+        c_hi = c;
+      }
+    }
+    (void)exact;
+    thr = (uint32_t)lo;
   }
-  int pos = 0;
-  int eq_taken = 0;
-  const bool all = m >= ncand;
-  const bool some = m > 0 && m < ncand;
+  // keys above thr are kept; of the keys equal to thr, the take_eq lowest ids
+  int above = 0, eqc = 0;
 #pragma unroll
   for (int k = 0; k < KPL; ++k) {
-    if (k * 32 >= Nb) break;
-    const int j = k * 32 + lane;
-    const bool in_range = j < Nb;
-    const bool is_sink = in_range && j < nsink;
-    const bool above = in_range && !is_sink && (all ? key[k] != 0u : key[k] > thr);
-    const bool eq = in_range && !is_sink && some && key[k] == thr;
-    const uint32_t eqmask = __ballot_sync(0xffffffffu, eq);
-    const int eq_rank = eq_taken + __popc(eqmask & ((1u << lane) - 1u));
-    const bool take = is_sink || above || (eq && eq_rank < take_eq);
-    eq_taken += __popc(eqmask);
-    const uint32_t tmask = __ballot_sync(0xffffffffu, take);
-    const int p = pos + __popc(tmask & ((1u << lane) - 1u));
-    if (take && p < kmax) out[p] = j;
-    pos += __popc(tmask);
+    above += key[k] > thr;
+    eqc += key[k] == thr;
+  }
+  above = (int)__reduce_add_sync(0xffffffffu, (uint32_t)above);
+  eqc = (int)__reduce_add_sync(0xffffffffu, (uint32_t)eqc);
+  const bool all = m >= ncand;
+  const bool some = m > 0 && m < ncand;
+  const int take_eq = some ? m - above : 0;
+  int pos = 0;
+  if (!some || take_eq == eqc) {
+    // every key equal to thr is kept (or none is): one ballot per 32 blocks
+#pragma unroll
+    for (int k = 0; k < KPL; ++k) {
+      if (k * 32 >= Nb) break;
+      const int j = k * 32 + lane;
+      const bool in_range = j < Nb;
+      const bool is_sink = in_range && j < nsink;
+      const bool cand = in_range && !is_sink && key[k] != 0u;
+      const bool take = is_sink || (cand && (all || (some && key[k] >= thr)));
+      const uint32_t tmask = __ballot_sync(0xffffffffu, take);
+      const int p = pos + __popc(tmask & ((1u << lane) - 1u));
+      if (take && p < kmax) out[p] = j;
+      pos += __popc(tmask);
+    }
+  } else {
+    int eq_taken = 0;
+#pragma unroll
+    for (int k = 0; k < KPL; ++k) {
+      if (k * 32 >= Nb) break;
+      const int j = k * 32 + lane;
+      const bool in_range = j < Nb;
+      const bool is_sink = in_range && j < nsink;
+      const bool gt = in_range && !is_sink && key[k] > thr;
+      const bool eq = in_range && !is_sink && key[k] == thr;
+      const uint32_t eqmask = __ballot_sync(0xffffffffu, eq);
+      const int eq_rank = eq_taken + __popc(eqmask & ((1u << lane) - 1u));
+      const bool take = is_sink || gt || (eq && eq_rank < take_eq);
+      eq_taken += __popc(eqmask);
+      const uint32_t tmask = __ballot_sync(0xffffffffu, take);
+      const int p = pos + __popc(tmask & ((1u << lane) - 1u));
+      if (take && p < kmax) out[p] = j;
+      pos += __popc(tmask);
+    }
   }
   for (int p = pos + lane; p < kmax; p += 32) out[p] = -1;
   if (lane == 0) *cnt_out = pos;
@@ -231,36 +380,51 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
 
 }  // namespace
 
-cudaError_t launch_pool(const void* qp, const void* kp, float* qbar, float* kbar, const Geo& g,
+cudaError_t launch_pool(const void* qp, const void* kp, __nv_bfloat16* q3, __nv_bfloat16* k3, const Geo& g,
                         cudaStream_t s) {
   int chunks = g.heads * g.D / 8;
   dim3 grid((chunks + kPoolThreads - 1) / kPoolThreads, g.Nb, g.B * 2);
-  pool_kernel<<<grid, kPoolThreads, 0, s>>>((const int4*)qp, (const int4*)kp, qbar, kbar, g,
-                                            chunks);
+  pool_kernel<<<grid, kPoolThreads, 0, s>>>((const int4*)qp, (const int4*)kp, q3, k3, g, chunks);
   return cudaGetLastError();
 }
 
+// 2-D view [3 * B*heads*Nb rows, D] of the bf16 parts; box 64 columns x 128 rows, 128-byte
+// swizzle (the K-major operand layout of the MMAs).
+static bool make_parts_map(CUtensorMap* m, const void* base, const Geo& g) {
+  EncodeTiledFn fn = tensor_map_encoder();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)g.D, (cuuint64_t)3 * g.B * g.heads * g.Nb};
+  cuuint64_t strides[1] = {(cuuint64_t)g.D * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kSTile};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D>
-cudaError_t launch_scores_d(const float* qbar, const float* kbar, float* scores, const Geo& g,
-                            float scale, cudaStream_t s) {
-  const int smem = 2 * D * kSPad * (int)sizeof(float);
+cudaError_t launch_scores_d(const __nv_bfloat16* q3, const __nv_bfloat16* k3, float* scores, const Geo& g,
+                            float scale, int32_t* status, cudaStream_t s) {
+  using C = ScoresCfg<D>;
+  CUtensorMap ta, tb;
+  if (!make_parts_map(&ta, q3, g) || !make_parts_map(&tb, k3, g)) return cudaErrorInvalidValue;
   static int configured_device = -1;  // one flag per instance (per D)
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(scores_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(scores_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
   dim3 grid((g.Nb + kSTile - 1) / kSTile, (g.Nb + kSTile - 1) / kSTile, g.B * g.heads);
-  scores_kernel<D><<<grid, 256, smem, s>>>(qbar, kbar, scores, g, scale);
+  scores_kernel<D><<<grid, kSThreads, C::kSmem, s>>>(ta, tb, scores, g, scale, status);
   return cudaGetLastError();
 }
 
-cudaError_t launch_scores(const float* qbar, const float* kbar, float* scores, const Geo& g,
-                          float scale, cudaStream_t s) {
-  if (g.D == 128) return launch_scores_d<128>(qbar, kbar, scores, g, scale, s);
-  return launch_scores_d<64>(qbar, kbar, scores, g, scale, s);
+cudaError_t launch_scores(const __nv_bfloat16* q3, const __nv_bfloat16* k3, float* scores, const Geo& g,
+                          float scale, int32_t* status, cudaStream_t s) {
+  if (g.D == 128) return launch_scores_d<128>(q3, k3, scores, g, scale, status, s);
+  return launch_scores_d<64>(q3, k3, scores, g, scale, status, s);
 }
 
 cudaError_t launch_topk(const float* scores, int32_t* idx, int32_t* cnt, int kmax, int kept,

@@ -10,8 +10,9 @@
 //
 // The array (kScratchBytes) exists on every GPU that loads this library, from module
 // load until the process exits.  Every call on a device shares it and it keeps the last
-// call's contents; nothing in it has to start at zero, because each call writes every
-// byte it reads (block means, then pooled scores) before reading it.  Calls whose work
+// call's contents.  Each call first clears the one word that must start at zero (its
+// status word) and writes every other byte it reads (the parts of the block means, then
+// the pooled scores) before reading it.  Calls whose work
 // overlaps on the GPU (on different streams, or different host threads, of the same
 // device) race on the array and must be serialised by the caller.
 #include <math.h>
@@ -47,8 +48,6 @@ int scratch_for_current_device(void** out) {
   return RF2_OK;
 }
 
-size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
@@ -70,21 +69,26 @@ extern "C" int rf2_predict_mask_noalloc(const void* qp, const void* kp, const rf
   int st = scratch_for_current_device(&base);
   if (st != RF2_OK) return st;
   const rf2::Geo geo = rf2::make_geo(*g);
-  const size_t means = (size_t)geo.B * geo.heads * geo.Nb * geo.D * sizeof(float);
+  // The same layout as the workspace of rf2_predict_mask: a status word, then the bf16
+  // parts of the block means and the pooled scores.
   unsigned char* p = static_cast<unsigned char*>(base);
-  float* qbar = reinterpret_cast<float*>(p);
-  float* kbar = reinterpret_cast<float*>(p + up(means));
-  float* scores = reinterpret_cast<float*>(p + 2 * up(means));
+  int32_t* status = reinterpret_cast<int32_t*>(p);
+  const rf2::MaskScratch m = rf2::mask_scratch_layout(geo, p + kAlign);
 
   cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = rf2::launch_pool(qp, kp, qbar, kbar, geo, s);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), s);
+  if (e == cudaSuccess) e = rf2::launch_pool(qp, kp, m.q3, m.k3, geo, s);
   if (e == cudaSuccess)
-    e = rf2::launch_scores(qbar, kbar, scores, geo, (float)(1.0 / sqrt((double)geo.D)), s);
+    e = rf2::launch_scores(m.q3, m.k3, m.scores, geo, (float)(1.0 / sqrt((double)geo.D)), status, s);
   if (e == cudaSuccess)
-    e = rf2::launch_topk(scores, idx, cnt, kmax, kept, sink ? geo.nbh * geo.nbw : 0, geo, s);
+    e = rf2::launch_topk(m.scores, idx, cnt, kmax, kept, sink ? geo.nbh * geo.nbw : 0, geo, s);
   if (e != cudaSuccess) return RF2_ERR_CUDA;
   if (flags & RF2_CHECKED) {
-    if (cudaStreamSynchronize(s) != cudaSuccess) return RF2_ERR_CUDA;
+    int32_t st_h = 0;
+    if (cudaMemcpyAsync(&st_h, status, sizeof(st_h), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return RF2_ERR_CUDA;
+    return st_h;
   }
   return RF2_OK;
 }

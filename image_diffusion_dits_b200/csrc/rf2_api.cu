@@ -52,25 +52,15 @@ int kept_of(const Geo& g, double sparsity, int sink, unsigned flags) {
 
 struct MaskWs {
   int32_t* status;
-  float* qbar;
-  float* kbar;
-  float* scores;
+  rf2::MaskScratch m;  // bf16 parts of the block means, pooled scores
   size_t bytes;
 };
 
 MaskWs mask_ws_layout(const Geo& g, uint8_t* base) {
   MaskWs w;
-  size_t off = 0;
-  w.status = reinterpret_cast<int32_t*>(base + off);
-  off += kAlign;
-  const size_t means = (size_t)g.B * g.heads * g.Nb * g.D * sizeof(float);
-  w.qbar = reinterpret_cast<float*>(base + off);
-  off += align_up(means);
-  w.kbar = reinterpret_cast<float*>(base + off);
-  off += align_up(means);
-  w.scores = reinterpret_cast<float*>(base + off);
-  off += align_up((size_t)g.B * g.heads * g.Nb * g.Nb * sizeof(float));
-  w.bytes = off;
+  w.status = reinterpret_cast<int32_t*>(base);
+  w.m = rf2::mask_scratch_layout(g, base + kAlign);
+  w.bytes = kAlign + align_up(w.m.bytes);
   return w;
 }
 
@@ -189,11 +179,11 @@ static int predict_mask_impl(const void* qp, const void* kp, const Geo& geo, dou
                              const MaskWs& w, cudaStream_t s) {
   const int kept = kept_of(geo, sparsity, sink, flags);
   log_geo("predict_mask", geo, kept);
-  cudaError_t e = rf2::launch_pool(qp, kp, w.qbar, w.kbar, geo, s);
+  cudaError_t e = rf2::launch_pool(qp, kp, w.m.q3, w.m.k3, geo, s);
   if (e == cudaSuccess)
-    e = rf2::launch_scores(w.qbar, w.kbar, w.scores, geo, (float)(1.0 / sqrt((double)geo.D)), s);
+    e = rf2::launch_scores(w.m.q3, w.m.k3, w.m.scores, geo, (float)(1.0 / sqrt((double)geo.D)), w.status, s);
   if (e == cudaSuccess)
-    e = rf2::launch_topk(w.scores, idx, cnt, kmax, kept, nsink_of(geo, sink), geo, s);
+    e = rf2::launch_topk(w.m.scores, idx, cnt, kmax, kept, nsink_of(geo, sink), geo, s);
   return cuda_status(e);
 }
 
@@ -211,10 +201,11 @@ int rf2_predict_mask(const void* qp, const void* kp, const rf2_geom* g, double s
   if (ws == nullptr || !aligned16(ws)) return ws == nullptr ? RF2_ERR_WORKSPACE : RF2_ERR_ALIGNMENT;
   MaskWs w = mask_ws_layout(geo, static_cast<uint8_t*>(ws));
   if (ws_bytes < w.bytes) return RF2_ERR_WORKSPACE;
+  if (cudaMemsetAsync(w.status, 0, sizeof(int32_t), (cudaStream_t)stream) != cudaSuccess) return RF2_ERR_CUDA;
   st = predict_mask_impl(qp, kp, geo, sparsity, sink, flags, idx, cnt, kmax, w,
                          (cudaStream_t)stream);
   if (st != RF2_OK) return st;
-  return finish_checked(flags, nullptr, (cudaStream_t)stream);
+  return finish_checked(flags, w.status, (cudaStream_t)stream);
 }
 
 int rf2_sparse_attn(const void* qp, const void* kp, const void* vp, const int32_t* idx,

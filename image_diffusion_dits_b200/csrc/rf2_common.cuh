@@ -1,6 +1,7 @@
 // Shared host/device definitions of the sm_100a block-sparse attention library.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -77,6 +78,34 @@ __host__ __device__ __forceinline__ void block_extent(const Geo& g, int j, int& 
   nw = min(g.ww, g.W - wb * g.ww);
 }
 
+// Scratch of the mask prediction (after the call's status word): the bf16 parts of the
+// block means of Q and K, then the pooled scores.  Shared by rf2_predict_mask and
+// rf2_predict_mask_noalloc.
+struct MaskScratch {
+  __nv_bfloat16* q3;
+  __nv_bfloat16* k3;
+  float* scores;
+  size_t bytes;
+};
+
+inline MaskScratch mask_scratch_layout(const Geo& g, unsigned char* base) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t parts = up((size_t)3 * g.B * g.heads * g.Nb * g.D * sizeof(__nv_bfloat16));
+  MaskScratch m;
+  m.q3 = reinterpret_cast<__nv_bfloat16*>(base);
+  m.k3 = reinterpret_cast<__nv_bfloat16*>(base + parts);
+  m.scores = reinterpret_cast<float*>(base + 2 * parts);
+  m.bytes = 2 * parts + up((size_t)g.B * g.heads * g.Nb * g.Nb * sizeof(float));
+  return m;
+}
+
+// cuTensorMapEncodeTiled from the driver (looked up once), or null if unavailable.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn tensor_map_encoder();
+
 // Device status word values (match rf2_status).
 constexpr int kStatusBadIndex = RF2_ERR_BAD_INDEX;
 constexpr int kStatusTimeout = RF2_ERR_TIMEOUT;
@@ -84,10 +113,14 @@ constexpr int kStatusTimeout = RF2_ERR_TIMEOUT;
 // Launchers (defined in the kernel files, called by the C ABI layer).
 cudaError_t launch_permute(const void* x, void* xp, const Geo& g, cudaStream_t s);
 cudaError_t launch_unpermute(const void* xp, void* x, const Geo& g, cudaStream_t s);
-cudaError_t launch_pool(const void* qp, const void* kp, float* qbar, float* kbar, const Geo& g,
+// Block means of Q and K, each written as three bf16 parts hi + mid + lo (about 24
+// significant bits together) in [3][B*heads*Nb][D] layout for the tensor-core scores.
+cudaError_t launch_pool(const void* qp, const void* kp, __nv_bfloat16* q3, __nv_bfloat16* k3, const Geo& g,
                         cudaStream_t s);
-cudaError_t launch_scores(const float* qbar, const float* kbar, float* scores, const Geo& g,
-                          float scale, cudaStream_t s);
+// Pooled scores s = qbar . kbar * scale from the bf16 parts (tcgen05); status (may be
+// null) receives RF2_ERR_TIMEOUT if a wait ran out.
+cudaError_t launch_scores(const __nv_bfloat16* q3, const __nv_bfloat16* k3, float* scores, const Geo& g,
+                          float scale, int32_t* status, cudaStream_t s);
 cudaError_t launch_topk(const float* scores, int32_t* idx, int32_t* cnt, int kmax, int kept,
                         int nsink, const Geo& g, cudaStream_t s);
 // Returns cudaErrorNotSupported when the shape has no kernel instance.
