@@ -376,26 +376,22 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-// 2^x on the FMA pipe, for x <= 64 (the softmax's arguments are <= 8): x = n + f with
-// n = round(x) taken from the low mantissa bits of x + 1.5*2^23 and f in [-0.5, 0.5];
-// 2^f from a cubic fitted here for minimum relative error on [-0.5, 0.5] (max relative
-// error 7.5e-5, far below the bf16 rounding of P); n is added to the exponent field.
-// Arguments below -125 (masked keys, -inf) give 2^-125, which is zero for P in bf16 and
-// negligible in the row sum.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  float p = fmaf(0.05517259240150452f, f, 0.24261370301246643f);
-  p = fmaf(p, f, 0.6932610273361206f);
-  p = fmaf(p, f, 0.9999278783798218f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^a0, 2^a1 on the exp2 unit in one packed f16 operation: the arguments are rounded to
+// f16 (nearest), the results widened back to fp32.  -inf gives 0; arguments below about
+// -24 underflow to 0.
+__device__ __forceinline__ void ex2_f16x2(float a0, float a1, float& p0, float& p1) {
+  uint32_t h2, e2;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h2) : "f"(a1), "f"(a0));  // first source -> upper half
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(e2) : "r"(h2));
+  asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tcvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
+      : "=f"(p0), "=f"(p1)
+      : "r"(e2));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
