@@ -87,8 +87,9 @@ def _cuda_bf16(t: torch.Tensor, name: str, shape) -> None:
         raise ValueError(f"{name}: expected contiguous bf16 {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
 
 
-def _flags(additive: bool, checked: bool) -> int:
-    return (RF2_SINK_ADDITIVE if additive else 0) | (RF2_CHECKED if checked else 0)
+def _flags(additive: bool, checked: bool, raster: bool = False) -> int:
+    return ((RF2_SINK_ADDITIVE if additive else 0) | (RF2_CHECKED if checked else 0) |
+            (_lib.RF2_RASTER if raster else 0))
 
 
 def permute(x: torch.Tensor, g: Geometry, out: Optional[torch.Tensor] = None) -> torch.Tensor:
@@ -131,10 +132,13 @@ def workspace_size(g: Geometry, sparsity: float, sink: bool, additive: bool = Fa
 def predict_mask(qp: torch.Tensor, kp: torch.Tensor, g: Geometry, sparsity: float, sink: bool,
                  additive: bool = False, kmax: Optional[int] = None, checked: bool = False,
                  ws: Optional[torch.Tensor] = None,
-                 out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Kept block lists idx [B, heads, Nb, kmax] (ascending, -1 padded) and counts."""
-    _cuda_bf16(qp, "qp", (g.B, g.Npad, g.heads, g.D))
-    _cuda_bf16(kp, "kp", (g.B, g.Npad, g.heads, g.D))
+                 out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None,
+                 raster: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Kept block lists idx [B, heads, Nb, kmax] (ascending, -1 padded) and counts.
+    qp, kp: window order [B, Npad, heads, D], or model order [B, N, heads, D] when raster."""
+    rows = g.N if raster else g.Npad
+    _cuda_bf16(qp, "qp", (g.B, rows, g.heads, g.D))
+    _cuda_bf16(kp, "kp", (g.B, rows, g.heads, g.D))
     k = kept_count(g, sparsity, sink, additive) if kmax is None else kmax
     if out is None:
         idx = torch.empty((g.B, g.heads, g.Nb, k), dtype=torch.int32, device=qp.device)
@@ -148,7 +152,7 @@ def predict_mask(qp: torch.Tensor, kp: torch.Tensor, g: Geometry, sparsity: floa
         ws = torch.empty(nbytes, dtype=torch.uint8, device=qp.device)
     cg = g.c()
     _check(library().rf2_predict_mask(qp.data_ptr(), kp.data_ptr(), ctypes.byref(cg), float(sparsity),
-                                      int(sink), _flags(additive, checked), idx.data_ptr(), cnt.data_ptr(),
+                                      int(sink), _flags(additive, checked, raster), idx.data_ptr(), cnt.data_ptr(),
                                       k, ws.data_ptr(), ws.numel(), _stream(qp)), "rf2_predict_mask")
     return idx, cnt
 
@@ -156,9 +160,12 @@ def predict_mask(qp: torch.Tensor, kp: torch.Tensor, g: Geometry, sparsity: floa
 def sparse_attn(qp: torch.Tensor, kp: torch.Tensor, vp: torch.Tensor, idx: torch.Tensor,
                 cnt: torch.Tensor, g: Geometry, scale: float = 0.0, checked: bool = False,
                 out: Optional[torch.Tensor] = None,
-                status: Optional[torch.Tensor] = None) -> torch.Tensor:
+                status: Optional[torch.Tensor] = None, raster: bool = False) -> torch.Tensor:
+    """O over the kept blocks; qp/kp/vp/out in window order [B, Npad, heads, D], or in
+    model order [B, N, heads, D] when raster."""
+    rows = g.N if raster else g.Npad
     for t, n in ((qp, "qp"), (kp, "kp"), (vp, "vp")):
-        _cuda_bf16(t, n, (g.B, g.Npad, g.heads, g.D))
+        _cuda_bf16(t, n, (g.B, rows, g.heads, g.D))
     if idx.dtype != torch.int32 or cnt.dtype != torch.int32 or not idx.is_contiguous():
         raise ValueError("idx and cnt must be contiguous int32")
     if out is None:
@@ -169,7 +176,7 @@ def sparse_attn(qp: torch.Tensor, kp: torch.Tensor, vp: torch.Tensor, idx: torch
     _check(library().rf2_sparse_attn(qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), idx.data_ptr(),
                                      cnt.data_ptr(), idx.shape[-1], ctypes.byref(cg), float(scale),
                                      out.data_ptr(), 0 if status is None else status.data_ptr(),
-                                     _flags(False, checked), _stream(qp)), "rf2_sparse_attn")
+                                     _flags(False, checked, raster), _stream(qp)), "rf2_sparse_attn")
     return out
 
 
@@ -177,7 +184,8 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Geometry, sp
               sink: bool = True, scale: float = 0.0, additive: bool = False,
               return_idx: bool = False, checked: bool = False,
               ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None):
-    """The whole RF2 path: permute -> mask -> block-sparse attention -> unpermute."""
+    """The whole RF2 path on model-order tensors: mask prediction, then block-sparse
+    attention; the window permutation is done by the kernels' gathers and scatters."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _cuda_bf16(t, n, (g.B, g.N, g.heads, g.D))
     nbytes = workspace_size(g, sparsity, sink, additive, attention=True)

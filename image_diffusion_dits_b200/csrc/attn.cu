@@ -87,13 +87,29 @@ struct Misc {
   int pad;
 };
 
-template <int D, int BLK>
+// Row r of query block i as a model-order token of batch b (RASTER), or -1 for a pad row.
+__device__ __forceinline__ long long window_row_token(const Geo& g, int i, int r) {
+  const int per_t = g.nbh * g.nbw;
+  const int tb = i / per_t, hb = (i - tb * per_t) / g.nbw, wb = i - tb * per_t - hb * g.nbw;
+  const int whw = g.wh * g.ww;
+  const int dt = r / whw, dh = (r - dt * whw) / g.ww, dw = r - dt * whw - dh * g.ww;
+  const int t = tb * g.wt + dt, h = hb * g.wh + dh, w = wb * g.ww + dw;
+  if (t >= g.T || h >= g.H || w >= g.W) return -1;
+  return ((long long)t * g.H + h) * g.W + w;
+}
+
+// RASTER: Q/K/V and O in model order [B, N, heads, D]: each window is one 5-D TMA box
+// (64 columns x 1 head x ww x wh x wt tokens; tokens past the grid arrive as zeros, the
+// same rows the window-order layout holds as zero pads) and O rows are written to their
+// tokens.  Otherwise window order [B, Npad, heads, D] through 3-D boxes.  The shared-
+// memory tiles are byte for byte the same in both layouts.
+template <int D, int BLK, bool RASTER>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const int32_t* __restrict__ idx,
                        const int32_t* __restrict__ cnt, int kmax,
                        __nv_bfloat16* __restrict__ op, Geo g, float scale_log2,
-                       int* __restrict__ status) {
+                       int* __restrict__ status, int b_base) {
   using C = Cfg<D, BLK>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -111,9 +127,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = tid & 31;
   const int qblk = blockIdx.x;
   const int head = blockIdx.y;
-  const int b = blockIdx.z;
+  const int b = b_base + (int)blockIdx.z;
   const long long row = ((long long)b * g.heads + head) * g.Nb + qblk;
   const long long brow0 = (long long)b * g.Npad;  // first row of batch b in the 3-D maps
+  // TMA box of block j: window-order rows (3-D) or window coordinates (5-D, per batch)
+  auto load_block = [&](uint32_t dst, const CUtensorMap* map, uint32_t barrier, int j, int rows) {
+#pragma unroll
+    for (int a = 0; a < D / 64; ++a) {
+      if constexpr (RASTER) {
+        const int per_t = g.nbh * g.nbw;
+        const int tb = j / per_t, hb = (j - tb * per_t) / g.nbw, wb = j - tb * per_t - hb * g.nbw;
+        ptx::tma_load_5d(dst + a * (rows * 128), map, barrier, a * 64, head, wb * g.ww, hb * g.wh, tb * g.wt);
+      } else {
+        ptx::tma_load_3d(dst + a * (rows * 128), map, barrier, a * 64, head, (int)(brow0 + (long long)j * BLK));
+      }
+    }
+  };
 
   // ---------------------------------------------------------------- setup
   if (warp == kMmaWarp) {
@@ -168,6 +197,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       atomicCAS(status, 0, kStatusBadIndex);
     if (lane == 0) misc->n = n_out;
   }
+  if constexpr (RASTER && BLK < kBM) {
+    // A window box fills BLK of the kBM Q rows; clear the rest once so that the unused
+    // S rows are finite (their outputs are never written).
+    for (int e = tid; e < C::kAtomsD * (kBM - BLK) * 8; e += kThreads) {
+      const int a = e / ((kBM - BLK) * 8), rem = e - a * (kBM - BLK) * 8;
+      reinterpret_cast<uint4*>(smem + C::kOffQ + a * (kBM * 128) + BLK * 128)[rem] = make_uint4(0, 0, 0, 0);
+    }
+    ptx::fence_proxy_async_smem();
+  }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
@@ -179,11 +217,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------------------ TMA producer: Q, K
       ptx::prefetch_tmap(&tq);
       ptx::prefetch_tmap(&tk);
-      ptx::mbar_arrive_expect_tx(bar(BAR_Q), C::kQBytes);
+      // Q tile: kBM rows per atom in shared memory; a window-order box covers all kBM
+      // rows (past a 64-token block: the next block's rows, never used), a window box BLK.
+      ptx::mbar_arrive_expect_tx(bar(BAR_Q), RASTER ? C::kAtomsD * BLK * 128 : C::kQBytes);
+      if constexpr (RASTER) {
+        load_block(sQ, &tq, bar(BAR_Q), qblk, kBM);
+      } else {
 #pragma unroll
-      for (int a = 0; a < C::kAtomsD; ++a)
-        ptx::tma_load_3d(sQ + a * (kBM * 128), &tq, bar(BAR_Q), a * 64, head,
-                         (int)(brow0 + (long long)qblk * BLK));
+        for (int a = 0; a < C::kAtomsD; ++a)
+          ptx::tma_load_3d(sQ + a * (kBM * 128), &tq, bar(BAR_Q), a * 64, head,
+                           (int)(brow0 + (long long)qblk * BLK));
+      }
       int issued[kKStages];
 #pragma unroll
       for (int s = 0; s < kKStages; ++s) issued[s] = -1;
@@ -193,11 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              status, kWaitLimitNs, kStatusTimeout))
           break;
         ptx::mbar_arrive_expect_tx(bar(BAR_KFULL + s), C::kKVBytes);
-        const int zrow = (int)(brow0 + (long long)list_s[i] * BLK);
-#pragma unroll
-        for (int a = 0; a < C::kAtomsD; ++a)
-          ptx::tma_load_3d(sK + s * C::kKVBytes + a * (BLK * 128), &tk, bar(BAR_KFULL + s), a * 64,
-                           head, zrow);
+        load_block(sK + s * C::kKVBytes, &tk, bar(BAR_KFULL + s), list_s[i], BLK);
         issued[s] = i;
       }
       if (*abort_flag) {
@@ -220,11 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              status, kWaitLimitNs, kStatusTimeout))
           break;
         ptx::mbar_arrive_expect_tx(bar(BAR_VFULL + s), C::kKVBytes);
-        const int zrow = (int)(brow0 + (long long)list_s[i] * BLK);
-#pragma unroll
-        for (int a = 0; a < C::kAtomsD; ++a)
-          ptx::tma_load_3d(sV + s * C::kKVBytes + a * (BLK * 128), &tv, bar(BAR_VFULL + s), a * 64,
-                           head, zrow);
+        load_block(sV + s * C::kKVBytes, &tv, bar(BAR_VFULL + s), list_s[i], BLK);
         issued[s] = i;
       }
       if (*abort_flag) {
@@ -476,8 +512,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float inv = den > 0.f ? 1.0f / den : 0.f;
         const float w0 = f0 * inv, w1 = f1 * inv;
         const bool use1 = n > 1;  // stream 1 holds at least one block
-        __nv_bfloat16* orow = op + ((brow0 + (long long)qblk * BLK + r) * g.heads + head) * (long long)D +
-                              st * (D / 2);
+        long long orow_idx;  // output row of query row r (negative: a pad row, not written)
+        if constexpr (RASTER) {
+          const long long n_tok = r < BLK ? window_row_token(g, qblk, r) : -1;
+          orow_idx = n_tok < 0 ? -1 : (long long)b * g.N + n_tok;
+        } else {
+          orow_idx = r < BLK ? brow0 + (long long)qblk * BLK + r : -1;
+        }
+        __nv_bfloat16* orow = op + (orow_idx * g.heads + head) * (long long)D + st * (D / 2);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
           const uint32_t col = (uint32_t)(st * (D / 2) + c * 32);
@@ -489,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) a1[e] = 0u;
           }
-          if (r < BLK) {
+          if (orow_idx >= 0) {
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               float o[8];
@@ -509,8 +551,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 4 && tid < BLK) {
     // No kept block: the row attends to nothing; write zeros.
-    __nv_bfloat16* orow = op + ((brow0 + (long long)qblk * BLK + tid) * g.heads + head) * (long long)D;
-    for (int v = 0; v < D / 8; ++v) reinterpret_cast<uint4*>(orow)[v] = make_uint4(0, 0, 0, 0);
+    long long orow_idx;
+    if constexpr (RASTER) {
+      const long long n_tok = window_row_token(g, qblk, tid);
+      orow_idx = n_tok < 0 ? -1 : (long long)b * g.N + n_tok;
+    } else {
+      orow_idx = brow0 + (long long)qblk * BLK + tid;
+    }
+    if (orow_idx >= 0) {
+      __nv_bfloat16* orow = op + (orow_idx * g.heads + head) * (long long)D;
+      for (int v = 0; v < D / 8; ++v) reinterpret_cast<uint4*>(orow)[v] = make_uint4(0, 0, 0, 0);
+    }
   }
 
   // ---------------------------------------------------------------- teardown
@@ -559,15 +610,29 @@ bool make_map(CUtensorMap* m, const void* base, const Geo& g, int rows) {
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int BLK>
+// 5-D view of one batch of a [B, N, heads, D] bf16 tensor in model order: dims (D, heads,
+// W, H, T); box = 64 columns x 1 head x one (ww, wh, wt) window, 128-byte swizzle.  Box
+// parts past W, H or T are zero filled.
+bool make_window_map(CUtensorMap* m, const void* base, const Geo& g) {
+  EncodeTiledFn fn = tensor_map_encoder();
+  if (fn == nullptr) return false;
+  const cuuint64_t row = (cuuint64_t)g.heads * g.D * 2;  // bytes per token
+  cuuint64_t dims[5] = {(cuuint64_t)g.D, (cuuint64_t)g.heads, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.T};
+  cuuint64_t strides[4] = {(cuuint64_t)g.D * 2, row, row * g.W, row * g.W * g.H};
+  cuuint32_t box[5] = {64, 1, (cuuint32_t)g.ww, (cuuint32_t)g.wh, (cuuint32_t)g.wt};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, int BLK, bool RASTER>
 cudaError_t launch_instance(const void* qp, const void* kp, const void* vp, const int32_t* idx,
                             const int32_t* cnt, int kmax, const Geo& g, float scale, void* op,
                             int32_t* status, cudaStream_t s) {
   using C = Cfg<D, BLK>;
-  CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, qp, g, kBM) || !make_map(&tk, kp, g, BLK) || !make_map(&tv, vp, g, BLK))
-    return cudaErrorInvalidValue;
-  auto kern = sparse_attn_kernel<D, BLK>;
+  auto kern = sparse_attn_kernel<D, BLK, RASTER>;
   static int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -576,27 +641,55 @@ cudaError_t launch_instance(const void* qp, const void* kp, const void* vp, cons
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  dim3 grid(g.Nb, g.heads, g.B);
   const float scale_log2 = scale * 1.4426950408889634f;  // log2(e)
-  kern<<<grid, kThreads, C::kSmem, s>>>(tq, tk, tv, idx, cnt, kmax,
-                                        reinterpret_cast<__nv_bfloat16*>(op), g, scale_log2,
-                                        status);
-  return cudaGetLastError();
+  if constexpr (RASTER) {
+    // one launch per batch: the 5-D maps address one batch's tokens
+    const size_t bstride = (size_t)g.N * g.heads * g.D * 2;
+    for (int b = 0; b < g.B; ++b) {
+      CUtensorMap tq, tk, tv;
+      if (!make_window_map(&tq, (const char*)qp + b * bstride, g) ||
+          !make_window_map(&tk, (const char*)kp + b * bstride, g) ||
+          !make_window_map(&tv, (const char*)vp + b * bstride, g))
+        return cudaErrorInvalidValue;
+      dim3 grid(g.Nb, g.heads, 1);
+      kern<<<grid, kThreads, C::kSmem, s>>>(tq, tk, tv, idx, cnt, kmax, reinterpret_cast<__nv_bfloat16*>(op), g,
+                                            scale_log2, status, b);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  } else {
+    CUtensorMap tq, tk, tv;
+    if (!make_map(&tq, qp, g, kBM) || !make_map(&tk, kp, g, BLK) || !make_map(&tv, vp, g, BLK))
+      return cudaErrorInvalidValue;
+    dim3 grid(g.Nb, g.heads, g.B);
+    kern<<<grid, kThreads, C::kSmem, s>>>(tq, tk, tv, idx, cnt, kmax, reinterpret_cast<__nv_bfloat16*>(op), g,
+                                          scale_log2, status, 0);
+    return cudaGetLastError();
+  }
+}
+
+template <int D, int BLK>
+cudaError_t launch_layout(const void* qp, const void* kp, const void* vp, const int32_t* idx, const int32_t* cnt,
+                          int kmax, const Geo& g, float scale, void* op, int32_t* status, bool raster,
+                          cudaStream_t s) {
+  if (raster) return launch_instance<D, BLK, true>(qp, kp, vp, idx, cnt, kmax, g, scale, op, status, s);
+  return launch_instance<D, BLK, false>(qp, kp, vp, idx, cnt, kmax, g, scale, op, status, s);
 }
 
 }  // namespace
 
 cudaError_t launch_sparse_attn(const void* qp, const void* kp, const void* vp,
                                const int32_t* idx, const int32_t* cnt, int kmax, const Geo& g,
-                               float scale, void* op, int32_t* status, cudaStream_t s) {
+                               float scale, void* op, int32_t* status, bool raster, cudaStream_t s) {
   if (g.D == 128 && g.blk == 128)
-    return launch_instance<128, 128>(qp, kp, vp, idx, cnt, kmax, g, scale, op, status, s);
+    return launch_layout<128, 128>(qp, kp, vp, idx, cnt, kmax, g, scale, op, status, raster, s);
   if (g.D == 64 && g.blk == 64)
-    return launch_instance<64, 64>(qp, kp, vp, idx, cnt, kmax, g, scale, op, status, s);
+    return launch_layout<64, 64>(qp, kp, vp, idx, cnt, kmax, g, scale, op, status, raster, s);
   if (g.D == 128 && g.blk == 64)
-    return launch_instance<128, 64>(qp, kp, vp, idx, cnt, kmax, g, scale, op, status, s);
+    return launch_layout<128, 64>(qp, kp, vp, idx, cnt, kmax, g, scale, op, status, raster, s);
   if (g.D == 64 && g.blk == 128)
-    return launch_instance<64, 128>(qp, kp, vp, idx, cnt, kmax, g, scale, op, status, s);
+    return launch_layout<64, 128>(qp, kp, vp, idx, cnt, kmax, g, scale, op, status, raster, s);
   return cudaErrorNotSupported;
 }
 

@@ -32,6 +32,9 @@ __device__ __forceinline__ void acc_bf16x8(float (&a)[8], const int4& v) {
   }
 }
 
+// RASTER: Q and K in model order [B, N, heads, D] (a window's rows are gathered line by
+// line, (dt, dh) lines of nw consecutive tokens); else in window order [B, Npad, heads, D].
+template <bool RASTER>
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const int4* __restrict__ qp,
                                                             const int4* __restrict__ kp,
                                                             __nv_bfloat16* __restrict__ q3,
@@ -42,16 +45,30 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const int4* __restri
   const int b = blockIdx.z >> 1;
   const int which = blockIdx.z & 1;
   if (c >= chunks) return;
-  const int4* src = (which ? kp : qp) + ((long long)b * g.Npad + (long long)j * g.blk) * chunks + c;
   int nt, nh, nw;
   block_extent(g, j, nt, nh, nw);
+  const int4* base = (which ? kp : qp) + c;
+  // first token of the window, and the row strides of its (dt, dh) lines
+  long long row0, t_stride, h_stride;
+  if (RASTER) {
+    const int per_t = g.nbh * g.nbw;
+    const int tb = j / per_t, hb = (j - tb * per_t) / g.nbw, wb = j - tb * per_t - hb * g.nbw;
+    row0 = (long long)b * g.N + ((long long)tb * g.wt * g.H + (long long)hb * g.wh) * g.W + (long long)wb * g.ww;
+    t_stride = (long long)g.H * g.W;
+    h_stride = g.W;
+  } else {
+    row0 = (long long)b * g.Npad + (long long)j * g.blk;
+    t_stride = (long long)g.wh * g.ww;
+    h_stride = g.ww;
+  }
+  const int4* src = base + row0 * chunks;
   float a[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) a[k] = 0.f;
   // Real rows of the window: (dt < nt, dh < nh, dw < nw); rows are row-major in the window.
   for (int dt = 0; dt < nt; ++dt) {
     for (int dh = 0; dh < nh; ++dh) {
-      const int4* rowp = src + (long long)((dt * g.wh + dh) * g.ww) * chunks;
+      const int4* rowp = src + (dt * t_stride + dh * h_stride) * chunks;
       int dw = 0;
       for (; dw + kPoolUnroll <= nw; dw += kPoolUnroll) {
         int4 v[kPoolUnroll];
@@ -381,10 +398,13 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
 }  // namespace
 
 cudaError_t launch_pool(const void* qp, const void* kp, __nv_bfloat16* q3, __nv_bfloat16* k3, const Geo& g,
-                        cudaStream_t s) {
+                        bool raster, cudaStream_t s) {
   int chunks = g.heads * g.D / 8;
   dim3 grid((chunks + kPoolThreads - 1) / kPoolThreads, g.Nb, g.B * 2);
-  pool_kernel<<<grid, kPoolThreads, 0, s>>>((const int4*)qp, (const int4*)kp, q3, k3, g, chunks);
+  if (raster)
+    pool_kernel<true><<<grid, kPoolThreads, 0, s>>>((const int4*)qp, (const int4*)kp, q3, k3, g, chunks);
+  else
+    pool_kernel<false><<<grid, kPoolThreads, 0, s>>>((const int4*)qp, (const int4*)kp, q3, k3, g, chunks);
   return cudaGetLastError();
 }
 

@@ -66,7 +66,6 @@ MaskWs mask_ws_layout(const Geo& g, uint8_t* base) {
 
 struct AttnWs {
   MaskWs mask;
-  void *qp, *kp, *vp, *op;
   int32_t *idx, *cnt;
   size_t bytes;
 };
@@ -75,11 +74,6 @@ AttnWs attn_ws_layout(const Geo& g, int kept, uint8_t* base) {
   AttnWs w;
   w.mask = mask_ws_layout(g, base);
   size_t off = w.mask.bytes;
-  const size_t t = align_up((size_t)g.B * g.Npad * g.heads * g.D * 2);
-  w.qp = base + off; off += t;
-  w.kp = base + off; off += t;
-  w.vp = base + off; off += t;
-  w.op = base + off; off += t;
   w.idx = reinterpret_cast<int32_t*>(base + off);
   off += align_up((size_t)g.B * g.heads * g.Nb * kept * sizeof(int32_t));
   w.cnt = reinterpret_cast<int32_t*>(base + off);
@@ -179,7 +173,7 @@ static int predict_mask_impl(const void* qp, const void* kp, const Geo& geo, dou
                              const MaskWs& w, cudaStream_t s) {
   const int kept = kept_of(geo, sparsity, sink, flags);
   log_geo("predict_mask", geo, kept);
-  cudaError_t e = rf2::launch_pool(qp, kp, w.m.q3, w.m.k3, geo, s);
+  cudaError_t e = rf2::launch_pool(qp, kp, w.m.q3, w.m.k3, geo, (flags & RF2_RASTER) != 0, s);
   if (e == cudaSuccess)
     e = rf2::launch_scores(w.m.q3, w.m.k3, w.m.scores, geo, (float)(1.0 / sqrt((double)geo.D)), w.status, s);
   if (e == cudaSuccess)
@@ -223,7 +217,7 @@ int rf2_sparse_attn(const void* qp, const void* kp, const void* vp, const int32_
   const float sc = scale == 0.f ? (float)(1.0 / sqrt((double)geo.D)) : scale;
   log_geo("sparse_attn", geo, kmax);
   cudaError_t e = rf2::launch_sparse_attn(qp, kp, vp, idx, cnt, kmax, geo, sc, op, status,
-                                          (cudaStream_t)stream);
+                                          (flags & RF2_RASTER) != 0, (cudaStream_t)stream);
   if (e == cudaErrorNotSupported) return RF2_ERR_UNSUPPORTED;
   if (e != cudaSuccess) return RF2_ERR_CUDA;
   return finish_checked(flags, status, (cudaStream_t)stream);
@@ -249,17 +243,13 @@ int rf2_attention(const void* q, const void* k, const void* v, const rf2_geom* g
   cudaStream_t s = (cudaStream_t)stream;
   const float sc = scale == 0.f ? (float)(1.0 / sqrt((double)geo.D)) : scale;
   log_geo("attention", geo, kept);
+  // Model-order tensors throughout: the kernels gather each window in place.
   cudaError_t e = cudaMemsetAsync(w.mask.status, 0, sizeof(int32_t), s);
-  if (e == cudaSuccess) e = rf2::launch_permute(q, w.qp, geo, s);
-  if (e == cudaSuccess) e = rf2::launch_permute(k, w.kp, geo, s);
-  if (e == cudaSuccess) e = rf2::launch_permute(v, w.vp, geo, s);
   if (e != cudaSuccess) return RF2_ERR_CUDA;
-  st = predict_mask_impl(w.qp, w.kp, geo, sparsity, sink, flags, w.idx, w.cnt, kept, w.mask, s);
+  st = predict_mask_impl(q, k, geo, sparsity, sink, flags | RF2_RASTER, w.idx, w.cnt, kept, w.mask, s);
   if (st != RF2_OK) return st;
-  e = rf2::launch_sparse_attn(w.qp, w.kp, w.vp, w.idx, w.cnt, kept, geo, sc, w.op,
-                              w.mask.status, s);
+  e = rf2::launch_sparse_attn(q, k, v, w.idx, w.cnt, kept, geo, sc, o, w.mask.status, true, s);
   if (e == cudaErrorNotSupported) return RF2_ERR_UNSUPPORTED;
-  if (e == cudaSuccess) e = rf2::launch_unpermute(w.op, o, geo, s);
   if (e == cudaSuccess && idx_out != nullptr)
     e = cudaMemcpyAsync(idx_out, w.idx, (size_t)geo.B * geo.heads * geo.Nb * kept * sizeof(int32_t),
                         cudaMemcpyDeviceToDevice, s);

@@ -115,17 +115,20 @@ cudaError_t launch_permute(const void* x, void* xp, const Geo& g, cudaStream_t s
 cudaError_t launch_unpermute(const void* xp, void* x, const Geo& g, cudaStream_t s);
 // Block means of Q and K, each written as three bf16 parts hi + mid + lo (about 24
 // significant bits together) in [3][B*heads*Nb][D] layout for the tensor-core scores.
+// raster: Q and K in model order [B, N, heads, D], else window order [B, Npad, heads, D].
 cudaError_t launch_pool(const void* qp, const void* kp, __nv_bfloat16* q3, __nv_bfloat16* k3, const Geo& g,
-                        cudaStream_t s);
+                        bool raster, cudaStream_t s);
 // Pooled scores s = qbar . kbar * scale from the bf16 parts (tcgen05); status (may be
 // null) receives RF2_ERR_TIMEOUT if a wait ran out.
 cudaError_t launch_scores(const __nv_bfloat16* q3, const __nv_bfloat16* k3, float* scores, const Geo& g,
                           float scale, int32_t* status, cudaStream_t s);
 cudaError_t launch_topk(const float* scores, int32_t* idx, int32_t* cnt, int kmax, int kept,
                         int nsink, const Geo& g, cudaStream_t s);
-// Returns cudaErrorNotSupported when the shape has no kernel instance.
+// Returns cudaErrorNotSupported when the shape has no kernel instance.  raster: Q/K/V
+// and O in model order [B, N, heads, D] (windows gathered and scattered in place), else
+// window order [B, Npad, heads, D].
 cudaError_t launch_sparse_attn(const void* qp, const void* kp, const void* vp,
                                const int32_t* idx, const int32_t* cnt, int kmax, const Geo& g,
-                               float scale, void* op, int32_t* status, cudaStream_t s);
+                               float scale, void* op, int32_t* status, bool raster, cudaStream_t s);
 
 }  // namespace rf2

@@ -60,7 +60,13 @@ enum rf2_flags {
      * in-budget reading: kept = max(ceil((1-s)*Nb - 1e-6) clamped to [1,Nb], |S|). */
     RF2_SINK_ADDITIVE = 1u,
     /* Wait for the call's work on `stream` and return the device status word. */
-    RF2_CHECKED = 2u
+    RF2_CHECKED = 2u,
+    /* rf2_predict_mask and rf2_sparse_attn: Q, K, V and O are in model order
+     * [B, N, heads, D] (the tensors rf2_permute would take) instead of window order
+     * [B, Npad, heads, D].  The kernels then gather each 3D window straight from model
+     * order (pad tokens read as zeros) and write O rows to their tokens; the results are
+     * those of the window-order call on rf2_permute'd inputs, bit for bit. */
+    RF2_RASTER = 4u
 };
 
 /* rf2_permute - 3D window permutation (mlsanity index page, Abstract, insight (2)
@@ -86,8 +92,8 @@ int rf2_kept_count(const rf2_geom* g, double sparsity, int sink, unsigned flags)
 
 /* rf2_workspace_size - bytes of device workspace that rf2_predict_mask (attention = 0)
  * or rf2_attention (attention = 1) needs for this geometry, sparsity and flags.  The
- * workspace holds the pooled block means, pooled scores, the kept lists (attention) and
- * the permuted Q/K/V/O copies (attention), plus a status word.  Returns 0 on a bad
+ * workspace holds a status word, the block means (three bf16 parts each), the pooled
+ * scores and, for rf2_attention, the kept lists and counts.  Returns 0 on a bad
  * argument. */
 size_t rf2_workspace_size(const rf2_geom* g, double sparsity, int sink, unsigned flags,
                           int attention);
@@ -96,9 +102,12 @@ size_t rf2_workspace_size(const rf2_geom* g, double sparsity, int sink, unsigned
  * Abstract, insight (1) "block-wise mean values as representative tokens for sparse mask
  * prediction" and insight (3) "first-frame sink").
  *   qp, kp : [B, Npad, heads, D] bf16, window order (read).  Pad positions are ignored.
+ *            With RF2_RASTER: [B, N, heads, D], model order.
  *   Steps: qbar_i, kbar_j = fp32 mean over the real tokens of each block, per head;
- *   s_ij = qbar_i . kbar_j / sqrt(D) (fp32); each row keeps the sink blocks plus the
- *   highest-scoring other blocks (ties to the lower id) up to rf2_kept_count.
+ *   s_ij = qbar_i . kbar_j / sqrt(D) with fp32 accumulation (on the tensor cores, from
+ *   each mean split into three bf16 parts; relative error about 1e-6); each row keeps
+ *   the sink blocks plus the highest-scoring other blocks (ties to the lower id) up to
+ *   rf2_kept_count.
  *   idx : [B, heads, Nb, kmax] int32 (written): ascending kept block ids, then -1.
  *   cnt : [B, heads, Nb] int32 (written): the kept count of each row.
  *   kmax >= rf2_kept_count(...) else RF2_ERR_INVALID_ARG.
@@ -129,9 +138,9 @@ int rf2_predict_mask(const void* qp, const void* kp, const rf2_geom* g, double s
  *   device current (cudaGetSymbolAddress); make that first call before any stream
  *   capture.
  *   Sharing: the array exists on every GPU that loads the library until the process
- *   exits, and all calls on a device share it.  Each call writes all the scratch it reads
- *   before reading it, so nothing needs clearing; calls that overlap on the GPU (other
- *   streams or host threads on the same device) race and must be serialised.
+ *   exits, and all calls on a device share it.  Each call clears its status word and
+ *   writes all the other scratch it reads before reading it; calls that overlap on the
+ *   GPU (other streams or host threads on the same device) race and must be serialised.
  * Errors: as rf2_predict_mask. */
 int rf2_predict_mask_noalloc(const void* qp, const void* kp, const rf2_geom* g,
                              double sparsity, int sink, unsigned flags, int32_t* idx,
@@ -144,9 +153,11 @@ int rf2_predict_mask_noalloc(const void* qp, const void* kp, const rf2_geom* g,
  *   S = idx[b, head, i, 0..cnt-1]; M = -inf on pad keys, 0 elsewhere.
  *   qp, kp, vp : [B, Npad, heads, D] bf16 (read).   op : [B, Npad, heads, D] bf16
  *   (written; pad query rows are written too, with values of no meaning).
+ *   With RF2_RASTER: qp, kp, vp, op are [B, N, heads, D] in model order; every row of op
+ *   is written.
  *   scale : softmax scale, > 0; 0 means 1/sqrt(D) (negative: RF2_ERR_INVALID_ARG).
  *   Softmax statistics and the accumulator
- *   are fp32; P is rounded to bf16 for the P.V product.
+ *   are fp32; exp2 is taken in f16 and P rounded to bf16 for the P.V product.
  *   status : optional device int32 (may be NULL); when given it must be zero on entry
  *   and receives RF2_ERR_BAD_INDEX / RF2_ERR_TIMEOUT if the kernel detects one
  *   (out-of-range ids are skipped, never dereferenced).  With RF2_CHECKED and a status
@@ -158,7 +169,9 @@ int rf2_sparse_attn(const void* qp, const void* kp, const void* vp, const int32_
                     int32_t* status, unsigned flags, void* stream);
 
 /* rf2_attention - the whole path (sciencestack page, Figure 1 "Workflow of
- * RainFusion2.0"): permute Q/K/V -> predict mask -> block-sparse attention -> unpermute.
+ * RainFusion2.0"): predict mask -> block-sparse attention, both on model-order tensors
+ * (the 3D window permutation and its inverse are done by the kernels' window gathers
+ * and row scatters, with no permuted copies).
  *   q, k, v : [B, N, heads, D] bf16 (read).   o : [B, N, heads, D] bf16 (written).
  *   idx_out : optional [B, heads, Nb, kept] int32 copy of the kept lists (may be NULL).
  *   ws, ws_bytes : device scratch of at least rf2_workspace_size(..., 1) bytes.

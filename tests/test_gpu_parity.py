@@ -257,3 +257,52 @@ def test_attention_is_deterministic():
     a = rf2.attention(q, k, v, g, 0.8, True)
     b = rf2.attention(q, k, v, g, 0.8, True)
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+# ----------------------------------------------------------------------------- model-order (raster) path
+
+@pytest.mark.parametrize("shape", RAGGED)
+def test_predict_mask_raster_equals_window_order(shape):
+    """Pooling straight from model order gives the same kept lists as pooling the
+    permuted tensors (same rows summed in the same order)."""
+    g, og = rf2.Geometry(**shape), O.geom(**shape)
+    q, k, _ = _rand_bits(g, 1300)
+    for s, sink in ((0.8, True), (0.5, False)):
+        a = rf2.predict_mask(to_dev(O.permute(q, og)), to_dev(O.permute(k, og)), g, s, sink, checked=True)
+        b = rf2.predict_mask(to_dev(q), to_dev(k), g, s, sink, checked=True, raster=True)
+        assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("name", SMALL + LARGE)
+def test_predict_mask_raster_workloads(name):
+    wl, g, og = _geoms(name)
+    q, k, _ = _inputs(name)
+    a = rf2.predict_mask(rf2.permute(to_dev(q), g), rf2.permute(to_dev(k), g), g, wl.sparsity, wl.sink,
+                         checked=True)
+    b = rf2.predict_mask(to_dev(q), to_dev(k), g, wl.sparsity, wl.sink, checked=True, raster=True)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("shape", RAGGED)
+def test_sparse_attn_raster_equals_window_order(shape):
+    """Window gathers and row scatters in model order give, bit for bit, the
+    window-order kernel's output on permuted tensors, unpermuted."""
+    g, og = rf2.Geometry(**shape), O.geom(**shape)
+    q, k, v = _rand_bits(g, 1400)
+    qf, kf = (bf16_bits_to_f64(O.permute(a, og)) for a in (q, k))
+    sel = O.predict_mask(qf, kf, og, 0.5, True)
+    idx = torch.from_numpy(sel.idx).cuda()
+    cnt = torch.full(sel.idx.shape[:3], sel.kept, dtype=torch.int32, device="cuda")
+    win = rf2.sparse_attn(*(to_dev(O.permute(a, og)) for a in (q, k, v)), idx, cnt, g, checked=True)
+    ras = rf2.sparse_attn(to_dev(q), to_dev(k), to_dev(v), idx, cnt, g, checked=True, raster=True)
+    assert torch.equal(rf2.unpermute(win, g).view(torch.int16), ras.view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["video480p", "wan720p"])
+def test_sparse_attn_raster_workloads(name):
+    wl, g, og = _geoms(name)
+    q, k, v = (to_dev(a) for a in _inputs(name))
+    idx, cnt = rf2.predict_mask(q, k, g, wl.sparsity, wl.sink, checked=True, raster=True)
+    win = rf2.sparse_attn(rf2.permute(q, g), rf2.permute(k, g), rf2.permute(v, g), idx, cnt, g, checked=True)
+    ras = rf2.sparse_attn(q, k, v, idx, cnt, g, checked=True, raster=True)
+    assert torch.equal(rf2.unpermute(win, g).view(torch.int16), ras.view(torch.int16))
