@@ -163,6 +163,43 @@ def test_sparse_attn_large_workloads_sampled_rows(name):
     print(name, stats)
 
 
+@pytest.mark.parametrize("sparsity", [0.0, 0.5, 0.7, 0.9])
+def test_sparse_attn_longvideo_sweep_sampled_rows(sparsity):
+    """The long-video sparsity sweep (960 blocks; 960 / 480 / 288 / 96 kept per row)."""
+    wl, g, og = _geoms("longvideo")
+    q, k, v = _inputs("longvideo")
+    rng = np.random.default_rng(int(sparsity * 100) + 3)
+    rows = {(0, int(rng.integers(og.heads)), int(rng.integers(og.Nb))) for _ in range(3)}
+    rows |= {(0, 0, 0), (0, og.heads - 1, og.Nb - 1)}
+    stats = _attn_case(g, og, q, k, v, sparsity, wl.sink, rows=sorted(rows))
+    print("longvideo", sparsity, stats)
+
+
+def test_attention_end_to_end_additive_sink():
+    """The sink-outside-the-budget reading (RF2_SINK_ADDITIVE) through the fused call."""
+    wl, g, og = _geoms("video480p")
+    q, k, v = _inputs("video480p")
+    out, idx = rf2.attention(to_dev(q), to_dev(k), to_dev(v), g, wl.sparsity, wl.sink, additive=True,
+                             return_idx=True, checked=True)
+    qf, kf, vf = (bf16_bits_to_f64(O.permute(a, og)) for a in (q, k, v))
+    sel = O.predict_mask(qf, kf, og, wl.sparsity, wl.sink, True)
+    gidx = idx.cpu().numpy()
+    compare_lists(gidx, np.full(gidx.shape[:3], sel.kept), sel)
+    got = to_f64(out)
+    tok = O.position_to_token(og)
+    got_rows, ref_rows = [], []
+    for h in range(og.heads):
+        for i in range(0, og.Nb, 7):
+            if not np.array_equal(gidx[0, h, i], sel.idx[0, h, i]):
+                continue
+            ref = O.attention_block(qf, kf, vf, og, 0, h, i, sel.idx[0, h, i], 1 / np.sqrt(og.D))
+            t = tok[i * og.blk:(i + 1) * og.blk]
+            keep = t >= 0
+            ref_rows.append(ref[keep])
+            got_rows.append(got[0, t[keep], h])
+    print("video480p additive", assert_close(np.concatenate(got_rows), np.concatenate(ref_rows), "additive"))
+
+
 def test_sparse_attn_zero_sparsity_is_dense_attention():
     shape = dict(B=1, heads=2, T=3, H=9, W=10, D=64, wt=1, wh=8, ww=8)
     g, og = rf2.Geometry(**shape), O.geom(**shape)

@@ -65,3 +65,20 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
     p = torch.empty(16, dtype=torch.uint8, device="cuda").data_ptr()
     st = lib.rf2_predict_mask_noalloc(p, p, ctypes.byref(cg), 0.8, 1, 0, p, p, 132, None)
     assert st == _lib.RF2_ERR_WORKSPACE
+
+
+def test_noalloc_model_order_matches_window_order():
+    """With RF2_RASTER the no-allocation call pools straight from model-order Q and K and
+    must give the same lists as rf2_predict_mask on the permuted tensors."""
+    wl = WORKLOADS["video480p"]
+    g = rf2.Geometry(**wl.geom())
+    q, k, _ = gen_qkv(wl)
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+    qd, kd = to_dev(q), to_dev(k)
+    kept = rf2.kept_count(g, wl.sparsity, wl.sink)
+    ref_idx, ref_cnt = rf2.predict_mask(rf2.permute(qd, g), rf2.permute(kd, g), g, wl.sparsity, wl.sink,
+                                        kmax=kept)
+    for _ in range(2):
+        idx, cnt = _noalloc(qd, kd, g, wl.sparsity, wl.sink, _lib.RF2_RASTER, kept)
+        torch.cuda.synchronize()
+        assert torch.equal(idx, ref_idx) and torch.equal(cnt, ref_cnt)
