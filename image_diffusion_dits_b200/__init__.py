@@ -205,5 +205,65 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Geometry, sp
     return (out, idx) if return_idx else out
 
 
+@dataclasses.dataclass(frozen=True)
+class Schedule:
+    """Step schedule of one generation (rf2_schedule_action): the leading dense_fraction of
+    the steps run dense (the pages keep the first 10 % dense), then a new mask is predicted
+    every predict_interval sparse steps (1: every step, as the online method does) and
+    reused in between."""
+
+    total_steps: int
+    dense_fraction: float = 0.1
+    predict_interval: int = 1
+
+    def action(self, step: int) -> int:
+        sc = _lib.Rf2Schedule(int(self.total_steps), float(self.dense_fraction), int(self.predict_interval))
+        a = library().rf2_schedule_action(ctypes.byref(sc), int(step))
+        if a < 0:
+            raise Rf2Error(-a, "rf2_schedule_action")
+        return a
+
+
+class StepAttention:
+    """Block-sparse attention of one generation under a Schedule, on model-order tensors:
+    dense steps attend to every block, predict steps run the mask prediction of their layer
+    and attend with it, reuse steps attend with the layer's last predicted lists.  Every
+    step runs on the library's kernels (rf2_predict_mask, rf2_sparse_attn with RF2_RASTER)."""
+
+    def __init__(self, g: Geometry, sparsity: float, sink: bool = True, schedule: Optional[Schedule] = None,
+                 additive: bool = False):
+        self.g, self.sparsity, self.sink, self.additive = g, float(sparsity), bool(sink), bool(additive)
+        self.schedule = schedule if schedule is not None else Schedule(1, 0.0, 1)
+        self.kept = kept_count(g, sparsity, sink, additive)
+        self._lists = {}   # layer -> (idx, cnt) of its last prediction
+        self._dense = None
+        self._ws = None
+
+    def lists(self, layer):
+        """The kept lists (idx, cnt) the layer's last predict step produced."""
+        return self._lists[layer]
+
+    def __call__(self, layer, step: int, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        g = self.g
+        act = self.schedule.action(step)
+        if act == _lib.RF2_STEP_DENSE:
+            if self._dense is None:
+                idx = torch.arange(g.Nb, dtype=torch.int32, device=q.device).expand(g.B, g.heads, g.Nb, g.Nb)
+                cnt = torch.full((g.B, g.heads, g.Nb), g.Nb, dtype=torch.int32, device=q.device)
+                self._dense = (idx.contiguous(), cnt)
+            return sparse_attn(q, k, v, *self._dense, g, out=out, raster=True)
+        if act == _lib.RF2_STEP_PREDICT:
+            if self._ws is None:
+                self._ws = torch.empty(workspace_size(g, self.sparsity, self.sink, self.additive, attention=False),
+                                       dtype=torch.uint8, device=q.device)
+            buf = self._lists.get(layer)
+            self._lists[layer] = predict_mask(q, k, g, self.sparsity, self.sink, self.additive, kmax=self.kept,
+                                              ws=self._ws, out=buf, raster=True)
+        elif layer not in self._lists:
+            raise RuntimeError(f"step {step} reuses the mask of layer {layer!r}, which has none predicted yet")
+        return sparse_attn(q, k, v, *self._lists[layer], g, out=out, raster=True)
+
+
 def default_scale(D: int) -> float:
     return 1.0 / math.sqrt(D)

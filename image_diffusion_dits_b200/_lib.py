@@ -31,8 +31,19 @@ EXPORTS = (
     "rf2_predict_mask_noalloc",
     "rf2_sparse_attn",
     "rf2_attention",
+    "rf2_schedule_action",
     "rf2_status_string",
 )
+
+
+RF2_STEP_DENSE = 0
+RF2_STEP_PREDICT = 1
+RF2_STEP_REUSE = 2
+
+
+class Rf2Schedule(ctypes.Structure):
+    _fields_ = [("total_steps", ctypes.c_int), ("dense_fraction", ctypes.c_double),
+                ("predict_interval", ctypes.c_int)]
 
 
 class Rf2Geom(ctypes.Structure):
@@ -57,6 +68,7 @@ _SIGS = {
                                        _vp, _i32p, ctypes.c_uint, _vp]),
     "rf2_attention": (ctypes.c_int, [_vp, _vp, _vp, _gp, ctypes.c_double, ctypes.c_int, ctypes.c_float,
                                      _vp, _i32p, _vp, ctypes.c_size_t, ctypes.c_uint, _vp]),
+    "rf2_schedule_action": (ctypes.c_int, [ctypes.POINTER(Rf2Schedule), ctypes.c_int]),
     "rf2_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
 

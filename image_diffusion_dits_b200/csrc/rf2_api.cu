@@ -132,6 +132,18 @@ const char* rf2_status_string(int status) {
   }
 }
 
+int rf2_schedule_action(const rf2_schedule* sc, int step) {
+  if (sc == nullptr || sc->total_steps < 1 || sc->predict_interval < 1 ||
+      !(sc->dense_fraction >= 0.0 && sc->dense_fraction <= 1.0))
+    return -RF2_ERR_INVALID_ARG;
+  if (step < 0 || step >= sc->total_steps) return -RF2_ERR_INVALID_ARG;
+  long long n_dense = (long long)ceil(sc->dense_fraction * (double)sc->total_steps - 1e-6);
+  if (n_dense < 0) n_dense = 0;
+  if (n_dense > sc->total_steps) n_dense = sc->total_steps;
+  if (step < n_dense) return RF2_STEP_DENSE;
+  return ((step - n_dense) % sc->predict_interval == 0) ? RF2_STEP_PREDICT : RF2_STEP_REUSE;
+}
+
 int rf2_permute(const void* x, void* xp, const rf2_geom* g, void* stream) {
   int st = check_geom(g);
   if (st != RF2_OK) return st;

@@ -180,6 +180,29 @@ int rf2_attention(const void* q, const void* k, const void* v, const rf2_geom* g
                   double sparsity, int sink, float scale, void* o, int32_t* idx_out,
                   void* ws, size_t ws_bytes, unsigned flags, void* stream);
 
+/* Step schedule of the attention calls of one generation.  RainFusion v1 keeps the first
+ * 10 % of the diffusion timesteps dense (pith.science review, "Free parameters": dense
+ * timestep fraction); RainFusion2.0 predicts its mask online, on every step.  Reusing a
+ * predicted mask for a few steps is a deployment option the pages do not describe. */
+typedef struct rf2_schedule {
+    int total_steps;        /* diffusion steps of one generation, >= 1                    */
+    double dense_fraction;  /* leading fraction of steps run dense, in [0, 1] (pages: 0.1)  */
+    int predict_interval;   /* a new mask every this many sparse steps, >= 1 (1: every step) */
+} rf2_schedule;
+
+enum rf2_step_action {
+    RF2_STEP_DENSE = 0,    /* all blocks kept: rf2_attention with sparsity 0              */
+    RF2_STEP_PREDICT = 1,  /* predict a new mask (rf2_predict_mask) and attend with it     */
+    RF2_STEP_REUSE = 2     /* attend with the last predicted kept lists (rf2_sparse_attn)  */
+};
+
+/* rf2_schedule_action - the action of step `step` (0-based): the first
+ * ceil(dense_fraction * total_steps - 1e-6) steps are dense; after them a new mask is
+ * predicted on the first sparse step and every predict_interval-th one, and the steps in
+ * between reuse it.  Host only (no device work).  Returns an rf2_step_action or
+ * -RF2_ERR_INVALID_ARG on a bad schedule or a step outside [0, total_steps). */
+int rf2_schedule_action(const rf2_schedule* schedule, int step);
+
 /* rf2_status_string - static, human-readable text of a status code. */
 const char* rf2_status_string(int status);
 

@@ -34,6 +34,7 @@ Parity status of each function (what pins it, in tests/test_oracle.py):
   select_blocks                          : rank-count brute force, planted orderings, invariants
   sparse_attention                       : dense brute force at 0% sparsity, torch SDPA (fp64),
                                            explicit -inf masked dense attention, closed forms
+  schedule_action                        : hand-worked step tables (tests/golden/schedule_actions.txt)
 The end-to-end RF2 numbers themselves are not printed on the pages (no worked example),
 so the method's outputs beyond these pins are "parity unpinned by the pages".
 """
@@ -346,3 +347,27 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, g: Geom, sparsity: fl
     sel = predict_mask(qp, kp, g, sparsity, sink, sink_additive)
     op = sparse_attention(qp, kp, vp, sel.idx, g, scale)
     return unpermute(op, g), sel
+
+
+# ----------------------------------------------------------------------------- step schedule
+
+DENSE, PREDICT, REUSE = 0, 1, 2
+
+
+def schedule_action(total_steps: int, dense_fraction: float, predict_interval: int, step: int) -> int:
+    """What the attention of diffusion step `step` (0-based, of `total_steps`) runs.
+
+    The first ceil(dense_fraction * total_steps - 1e-6) steps are dense (RainFusion v1
+    keeps the first 10 % of the timesteps dense: pith.science review, "Free parameters",
+    dense timestep fraction).  After them a new mask is predicted on the first sparse step
+    and then on every `predict_interval`-th one; the steps in between reuse the last
+    predicted mask.  predict_interval = 1 predicts on every step, as the online method
+    does; larger values are a deployment option the pages do not describe."""
+    if total_steps < 1 or predict_interval < 1 or not (0.0 <= dense_fraction <= 1.0):
+        raise ValueError("bad schedule")
+    if not 0 <= step < total_steps:
+        raise ValueError("step outside the schedule")
+    n_dense = min(max(math.ceil(dense_fraction * total_steps - 1e-6), 0), total_steps)
+    if step < n_dense:
+        return DENSE
+    return PREDICT if (step - n_dense) % predict_interval == 0 else REUSE

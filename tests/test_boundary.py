@@ -132,3 +132,21 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros((1, g.N, g.heads, g.D), dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         rf2.permute(x, g)
+
+
+def test_schedule_action_matches_oracle_and_rejects_bad_input():
+    import oracle as O
+    lib = _lib.load()
+    for total in (1, 3, 10, 50):
+        for frac in (0.0, 0.1, 0.5, 1.0):
+            for interval in (1, 2, 4):
+                sc = _lib.Rf2Schedule(total, frac, interval)
+                for s in range(total):
+                    assert lib.rf2_schedule_action(ctypes.byref(sc), s) == O.schedule_action(total, frac, interval, s)
+    sc = _lib.Rf2Schedule(10, 0.1, 1)
+    assert lib.rf2_schedule_action(ctypes.byref(sc), 10) == -_lib.RF2_ERR_INVALID_ARG
+    assert lib.rf2_schedule_action(ctypes.byref(sc), -1) == -_lib.RF2_ERR_INVALID_ARG
+    for bad in (_lib.Rf2Schedule(0, 0.1, 1), _lib.Rf2Schedule(10, 1.5, 1), _lib.Rf2Schedule(10, 0.1, 0)):
+        assert lib.rf2_schedule_action(ctypes.byref(bad), 0) == -_lib.RF2_ERR_INVALID_ARG
+    assert lib.rf2_schedule_action(None, 0) == -_lib.RF2_ERR_INVALID_ARG
+    assert rf2.Schedule(50, 0.1, 5).action(5) == _lib.RF2_STEP_PREDICT

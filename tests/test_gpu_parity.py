@@ -343,3 +343,36 @@ def test_sparse_attn_raster_workloads(name):
     win = rf2.sparse_attn(rf2.permute(q, g), rf2.permute(k, g), rf2.permute(v, g), idx, cnt, g, checked=True)
     ras = rf2.sparse_attn(q, k, v, idx, cnt, g, checked=True, raster=True)
     assert torch.equal(rf2.unpermute(win, g).view(torch.int16), ras.view(torch.int16))
+
+
+# ----------------------------------------------------------------------------- step schedule
+
+def test_step_attention_follows_its_schedule():
+    """Dense steps equal the fused call at 0 % sparsity, predict steps equal the fused
+    call at the target sparsity, reuse steps attend with the layer's last predicted lists
+    (bit for bit), and every layer keeps its own lists."""
+    wl, g, og = _geoms("video480p")
+    sched = rf2.Schedule(total_steps=10, dense_fraction=0.1, predict_interval=3)   # D P R R P R R P R R
+    sa = rf2.StepAttention(g, 0.5, wl.sink, schedule=sched)
+    inputs = {}
+    for layer in (0, 1):
+        for step in range(3):
+            inputs[layer, step] = [to_dev(gen_tensor(g.B, g.T, g.H, g.W, g.heads, g.D, 7000 + 100 * layer + 10 * step + i))
+                                   for i in range(3)]
+    same = lambda a, b: torch.equal(a.view(torch.int16), b.view(torch.int16))
+    for layer in (0, 1):
+        q, k, v = inputs[layer, 0]
+        assert same(sa(layer, 0, q, k, v), rf2.attention(q, k, v, g, 0.0, wl.sink))          # dense
+    for layer in (0, 1):
+        q, k, v = inputs[layer, 1]
+        assert same(sa(layer, 1, q, k, v), rf2.attention(q, k, v, g, 0.5, wl.sink))          # predict
+    for layer in (0, 1):
+        q, k, v = inputs[layer, 2]
+        idx, cnt = sa.lists(layer)
+        ref = rf2.sparse_attn(q, k, v, idx, cnt, g, raster=True)
+        assert same(sa(layer, 2, q, k, v), ref)                                               # reuse
+        q1, k1, _ = inputs[layer, 1]
+        i1, c1 = rf2.predict_mask(q1, k1, g, 0.5, wl.sink, raster=True)
+        assert torch.equal(idx, i1) and torch.equal(cnt, c1)   # the lists of that layer's predict step
+    with pytest.raises(RuntimeError):
+        rf2.StepAttention(g, 0.5, wl.sink, schedule=sched)(0, 2, *inputs[0, 2])               # reuse before predict

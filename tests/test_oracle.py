@@ -305,3 +305,38 @@ def test_generator_is_seeded_and_structured():
     np.testing.assert_array_equal(a, b)
     x = bf16_bits_to_f64(a)
     assert abs(x.mean()) < 0.2 and 0.9 < x.std() < 1.4
+
+
+# ----------------------------------------------------------------------------- step schedule
+
+def _golden_schedules():
+    path = os.path.join(os.path.dirname(__file__), "golden", "schedule_actions.txt")
+    rows = []
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        total, frac, interval, acts = line.split()
+        rows.append((int(total), float(frac), int(interval), acts))
+    return rows
+
+
+def test_schedule_matches_hand_worked_tables():
+    code = {O.DENSE: "D", O.PREDICT: "P", O.REUSE: "R"}
+    for total, frac, interval, acts in _golden_schedules():
+        assert len(acts) == total
+        got = "".join(code[O.schedule_action(total, frac, interval, s)] for s in range(total))
+        assert got == acts, (total, frac, interval)
+
+
+def test_schedule_invariants():
+    for total in (1, 2, 7, 30, 50, 100):
+        for frac in (0.0, 0.05, 0.1, 0.33, 1.0):
+            for interval in (1, 2, 3, 5):
+                acts = [O.schedule_action(total, frac, interval, s) for s in range(total)]
+                n_dense = sum(a == O.DENSE for a in acts)
+                assert n_dense == min(total, math.ceil(frac * total - 1e-6))
+                assert all(a == O.DENSE for a in acts[:n_dense])          # dense steps lead
+                if n_dense < total:
+                    assert acts[n_dense] == O.PREDICT                     # a mask exists before reuse
+                assert (O.REUSE in acts) == (interval > 1 and total - n_dense > 1)
