@@ -34,7 +34,11 @@ class Rf2Error(RuntimeError):
 
 @dataclasses.dataclass(frozen=True)
 class Geometry:
-    """Shape of one attention call: batch, heads, token grid, head_dim, 3D window."""
+    """Shape of one attention call: batch, heads, token grid, head_dim, 3D window.
+
+    no_permute selects the "without 3D permutation" ablation (RF2_NO_PERMUTE): blocks of
+    blk = wt*wh*ww consecutive raster tokens instead of 3D windows, and a sink of the
+    blocks that hold frame 0."""
 
     B: int
     heads: int
@@ -45,6 +49,7 @@ class Geometry:
     wt: int
     wh: int
     ww: int
+    no_permute: bool = False
 
     @property
     def N(self) -> int:
@@ -57,7 +62,13 @@ class Geometry:
     @property
     def Nb(self) -> int:
         c = lambda a, b: -(-a // b)
+        if self.no_permute:
+            return c(self.N, self.blk)
         return c(self.T, self.wt) * c(self.H, self.wh) * c(self.W, self.ww)
+
+    @property
+    def flags(self) -> int:
+        return _lib.RF2_NO_PERMUTE if self.no_permute else 0
 
     @property
     def Npad(self) -> int:
@@ -87,12 +98,18 @@ def _cuda_bf16(t: torch.Tensor, name: str, shape) -> None:
         raise ValueError(f"{name}: expected contiguous bf16 {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
 
 
-def _flags(additive: bool, checked: bool, raster: bool = False) -> int:
+def _flags(g: Geometry, additive: bool, checked: bool, raster: bool = False) -> int:
     return ((RF2_SINK_ADDITIVE if additive else 0) | (RF2_CHECKED if checked else 0) |
-            (_lib.RF2_RASTER if raster else 0))
+            (_lib.RF2_RASTER if raster else 0) | g.flags)
+
+
+def _windows_only(g: Geometry, where: str) -> None:
+    if g.no_permute:
+        raise ValueError(f"{where}: a no_permute geometry has no window permutation")
 
 
 def permute(x: torch.Tensor, g: Geometry, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _windows_only(g, "permute")
     _cuda_bf16(x, "x", (g.B, g.N, g.heads, g.D))
     if out is None:
         out = torch.empty((g.B, g.Npad, g.heads, g.D), dtype=torch.bfloat16, device=x.device)
@@ -102,6 +119,7 @@ def permute(x: torch.Tensor, g: Geometry, out: Optional[torch.Tensor] = None) ->
 
 
 def unpermute(xp: torch.Tensor, g: Geometry, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _windows_only(g, "unpermute")
     _cuda_bf16(xp, "xp", (g.B, g.Npad, g.heads, g.D))
     if out is None:
         out = torch.empty((g.B, g.N, g.heads, g.D), dtype=torch.bfloat16, device=xp.device)
@@ -113,7 +131,7 @@ def unpermute(xp: torch.Tensor, g: Geometry, out: Optional[torch.Tensor] = None)
 
 def kept_count(g: Geometry, sparsity: float, sink: bool, additive: bool = False) -> int:
     cg = g.c()
-    k = library().rf2_kept_count(ctypes.byref(cg), float(sparsity), int(sink), _flags(additive, False))
+    k = library().rf2_kept_count(ctypes.byref(cg), float(sparsity), int(sink), _flags(g, additive, False))
     if k < 0:
         raise Rf2Error(-k, "rf2_kept_count")
     return k
@@ -123,7 +141,7 @@ def workspace_size(g: Geometry, sparsity: float, sink: bool, additive: bool = Fa
                    attention: bool = True) -> int:
     cg = g.c()
     n = library().rf2_workspace_size(ctypes.byref(cg), float(sparsity), int(sink),
-                                     _flags(additive, False), int(attention))
+                                     _flags(g, additive, False), int(attention))
     if n == 0:
         raise Rf2Error(_lib.RF2_ERR_INVALID_ARG, "rf2_workspace_size")
     return n
@@ -152,7 +170,7 @@ def predict_mask(qp: torch.Tensor, kp: torch.Tensor, g: Geometry, sparsity: floa
         ws = torch.empty(nbytes, dtype=torch.uint8, device=qp.device)
     cg = g.c()
     _check(library().rf2_predict_mask(qp.data_ptr(), kp.data_ptr(), ctypes.byref(cg), float(sparsity),
-                                      int(sink), _flags(additive, checked, raster), idx.data_ptr(), cnt.data_ptr(),
+                                      int(sink), _flags(g, additive, checked, raster), idx.data_ptr(), cnt.data_ptr(),
                                       k, ws.data_ptr(), ws.numel(), _stream(qp)), "rf2_predict_mask")
     return idx, cnt
 
@@ -176,7 +194,7 @@ def sparse_attn(qp: torch.Tensor, kp: torch.Tensor, vp: torch.Tensor, idx: torch
     _check(library().rf2_sparse_attn(qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), idx.data_ptr(),
                                      cnt.data_ptr(), idx.shape[-1], ctypes.byref(cg), float(scale),
                                      out.data_ptr(), 0 if status is None else status.data_ptr(),
-                                     _flags(False, checked, raster), _stream(qp)), "rf2_sparse_attn")
+                                     _flags(g, False, checked, raster), _stream(qp)), "rf2_sparse_attn")
     return out
 
 
@@ -201,7 +219,7 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Geometry, sp
     _check(library().rf2_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(cg),
                                    float(sparsity), int(sink), float(scale), out.data_ptr(),
                                    0 if idx is None else idx.data_ptr(), ws.data_ptr(), ws.numel(),
-                                   _flags(additive, checked), _stream(q)), "rf2_attention")
+                                   _flags(g, additive, checked), _stream(q)), "rf2_attention")
     return (out, idx) if return_idx else out
 
 

@@ -19,6 +19,7 @@ RF2_ERR_CUDA = 7
 RF2_SINK_ADDITIVE = 1
 RF2_CHECKED = 2
 RF2_RASTER = 4
+RF2_NO_PERMUTE = 8
 RF2_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 # Every symbol include/rf2.h declares.

@@ -68,7 +68,7 @@ extern "C" int rf2_predict_mask_noalloc(const void* qp, const void* kp, const rf
   void* base = nullptr;
   int st = scratch_for_current_device(&base);
   if (st != RF2_OK) return st;
-  const rf2::Geo geo = rf2::make_geo(*g);
+  const rf2::Geo geo = rf2::make_call_geo(*g, flags);
   // The same layout as the workspace of rf2_predict_mask: a status word, then the bf16
   // parts of the block means and the pooled scores.
   unsigned char* p = static_cast<unsigned char*>(base);
@@ -81,7 +81,7 @@ extern "C" int rf2_predict_mask_noalloc(const void* qp, const void* kp, const rf
   if (e == cudaSuccess)
     e = rf2::launch_scores(m.q3, m.k3, m.scores, geo, (float)(1.0 / sqrt((double)geo.D)), status, s);
   if (e == cudaSuccess)
-    e = rf2::launch_topk(m.scores, idx, cnt, kmax, kept, sink ? geo.nbh * geo.nbw : 0, geo, s);
+    e = rf2::launch_topk(m.scores, idx, cnt, kmax, kept, sink ? geo.nsink : 0, geo, s);
   if (e != cudaSuccess) return RF2_ERR_CUDA;
   if (flags & RF2_CHECKED) {
     int32_t st_h = 0;

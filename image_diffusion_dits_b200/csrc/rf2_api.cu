@@ -17,7 +17,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int check_geom(const rf2_geom* g) {
+int check_geom(const rf2_geom* g, unsigned flags = 0) {
   if (g == nullptr) return RF2_ERR_INVALID_ARG;
   if (g->B < 1 || g->heads < 1 || g->T < 1 || g->H < 1 || g->W < 1 || g->wt < 1 || g->wh < 1 ||
       g->ww < 1 || g->D < 1)
@@ -25,13 +25,15 @@ int check_geom(const rf2_geom* g) {
   if (g->D != 64 && g->D != 128) return RF2_ERR_UNSUPPORTED;
   const long long blk = (long long)g->wt * g->wh * g->ww;
   if (blk != 64 && blk != 128) return RF2_ERR_UNSUPPORTED;
-  Geo o = rf2::make_geo(*g);
+  const long long n = (long long)g->T * g->H * g->W;
+  if ((long long)g->B * (n + blk) >= (1ll << 31)) return RF2_ERR_UNSUPPORTED;  // TMA coordinates
+  Geo o = rf2::make_call_geo(*g, flags);
   if (o.Nb > 1024) return RF2_ERR_UNSUPPORTED;                  // kept lists live in smem
   if ((long long)o.B * o.Npad >= (1ll << 31)) return RF2_ERR_UNSUPPORTED;  // TMA coordinates
   return RF2_OK;
 }
 
-int nsink_of(const Geo& g, int sink) { return sink ? g.nbh * g.nbw : 0; }
+int nsink_of(const Geo& g, int sink) { return sink ? g.nsink : 0; }
 
 // Kept blocks per row (both sides of the sink reading).  Every block holds at least one
 // real token (padding is less than one window per axis), so all Nb blocks are valid.
@@ -165,17 +167,17 @@ int rf2_unpermute(const void* xp, void* x, const rf2_geom* g, void* stream) {
 }
 
 int rf2_kept_count(const rf2_geom* g, double sparsity, int sink, unsigned flags) {
-  int st = check_geom(g);
+  int st = check_geom(g, flags);
   if (st != RF2_OK) return -st;
   if (!(sparsity >= 0.0 && sparsity <= 1.0)) return -RF2_ERR_INVALID_ARG;
-  return kept_of(rf2::make_geo(*g), sparsity, sink, flags);
+  return kept_of(rf2::make_call_geo(*g, flags), sparsity, sink, flags);
 }
 
 size_t rf2_workspace_size(const rf2_geom* g, double sparsity, int sink, unsigned flags,
                           int attention) {
-  if (check_geom(g) != RF2_OK) return 0;
+  if (check_geom(g, flags) != RF2_OK) return 0;
   if (!(sparsity >= 0.0 && sparsity <= 1.0)) return 0;
-  Geo geo = rf2::make_geo(*g);
+  Geo geo = rf2::make_call_geo(*g, flags);
   if (!attention) return mask_ws_layout(geo, nullptr).bytes;
   return attn_ws_layout(geo, kept_of(geo, sparsity, sink, flags), nullptr).bytes;
 }
@@ -196,13 +198,13 @@ static int predict_mask_impl(const void* qp, const void* kp, const Geo& geo, dou
 int rf2_predict_mask(const void* qp, const void* kp, const rf2_geom* g, double sparsity, int sink,
                      unsigned flags, int32_t* idx, int32_t* cnt, int kmax, void* ws,
                      size_t ws_bytes, void* stream) {
-  int st = check_geom(g);
+  int st = check_geom(g, flags);
   if (st != RF2_OK) return st;
   if (!(sparsity >= 0.0 && sparsity <= 1.0)) return RF2_ERR_INVALID_ARG;
   if (qp == nullptr || kp == nullptr || idx == nullptr || cnt == nullptr) return RF2_ERR_INVALID_ARG;
   if (!aligned16(qp) || !aligned16(kp) || !aligned16(idx) || !aligned16(cnt))
     return RF2_ERR_ALIGNMENT;
-  Geo geo = rf2::make_geo(*g);
+  Geo geo = rf2::make_call_geo(*g, flags);
   if (kmax < kept_of(geo, sparsity, sink, flags)) return RF2_ERR_INVALID_ARG;
   if (ws == nullptr || !aligned16(ws)) return ws == nullptr ? RF2_ERR_WORKSPACE : RF2_ERR_ALIGNMENT;
   MaskWs w = mask_ws_layout(geo, static_cast<uint8_t*>(ws));
@@ -217,7 +219,7 @@ int rf2_predict_mask(const void* qp, const void* kp, const rf2_geom* g, double s
 int rf2_sparse_attn(const void* qp, const void* kp, const void* vp, const int32_t* idx,
                     const int32_t* cnt, int kmax, const rf2_geom* g, float scale, void* op,
                     int32_t* status, unsigned flags, void* stream) {
-  int st = check_geom(g);
+  int st = check_geom(g, flags);
   if (st != RF2_OK) return st;
   if (qp == nullptr || kp == nullptr || vp == nullptr || idx == nullptr || cnt == nullptr ||
       op == nullptr || kmax < 1 || !isfinite(scale) || scale < 0.f)
@@ -225,7 +227,7 @@ int rf2_sparse_attn(const void* qp, const void* kp, const void* vp, const int32_
   if (!aligned16(qp) || !aligned16(kp) || !aligned16(vp) || !aligned16(op) ||
       ((uintptr_t)idx & 3u) || ((uintptr_t)cnt & 3u) || ((uintptr_t)status & 3u))
     return RF2_ERR_ALIGNMENT;
-  Geo geo = rf2::make_geo(*g);
+  Geo geo = rf2::make_call_geo(*g, flags);
   const float sc = scale == 0.f ? (float)(1.0 / sqrt((double)geo.D)) : scale;
   log_geo("sparse_attn", geo, kmax);
   cudaError_t e = rf2::launch_sparse_attn(qp, kp, vp, idx, cnt, kmax, geo, sc, op, status,
@@ -238,7 +240,7 @@ int rf2_sparse_attn(const void* qp, const void* kp, const void* vp, const int32_
 int rf2_attention(const void* q, const void* k, const void* v, const rf2_geom* g, double sparsity,
                   int sink, float scale, void* o, int32_t* idx_out, void* ws, size_t ws_bytes,
                   unsigned flags, void* stream) {
-  int st = check_geom(g);
+  int st = check_geom(g, flags);
   if (st != RF2_OK) return st;
   if (!(sparsity >= 0.0 && sparsity <= 1.0) || !isfinite(scale) || scale < 0.f)
     return RF2_ERR_INVALID_ARG;
@@ -248,7 +250,7 @@ int rf2_attention(const void* q, const void* k, const void* v, const rf2_geom* g
     return RF2_ERR_ALIGNMENT;
   if (ws == nullptr) return RF2_ERR_WORKSPACE;
   if (!aligned16(ws)) return RF2_ERR_ALIGNMENT;
-  Geo geo = rf2::make_geo(*g);
+  Geo geo = rf2::make_call_geo(*g, flags);
   const int kept = kept_of(geo, sparsity, sink, flags);
   AttnWs w = attn_ws_layout(geo, kept, static_cast<uint8_t*>(ws));
   if (ws_bytes < w.bytes) return RF2_ERR_WORKSPACE;

@@ -19,6 +19,7 @@ struct Geo {
   int nbt, nbh, nbw;  // windows per axis
   int Nb, blk;        // blocks, tokens per block
   long long N, Npad;  // real tokens, padded tokens (per batch)
+  int nsink;          // blocks that hold a token of frame 0 (the first-frame sink)
 };
 
 inline Geo make_geo(const rf2_geom& g) {
@@ -32,6 +33,24 @@ inline Geo make_geo(const rf2_geom& g) {
   o.blk = g.wt * g.wh * g.ww;
   o.N = (long long)g.T * g.H * g.W;
   o.Npad = (long long)o.Nb * o.blk;
+  o.nsink = o.nbh * o.nbw;  // temporal window 0
+  return o;
+}
+
+// Geometry of a call with `flags`.  RF2_NO_PERMUTE ("without 3D permutation" ablation,
+// sciencestack page, Figure 3 (b)): blocks are blk consecutive raster tokens, i.e. the
+// flat grid (1, 1, N) cut into (1, 1, blk) windows; the sink is the blocks holding a
+// frame-0 token.  The caller checks that N fits an int (N < 2^31 follows from the
+// coordinate limit of the kernels).
+inline Geo make_call_geo(const rf2_geom& g, unsigned flags) {
+  if (!(flags & RF2_NO_PERMUTE)) return make_geo(g);
+  rf2_geom f = g;
+  f.T = 1; f.H = 1; f.W = g.T * g.H * g.W;
+  f.wt = 1; f.wh = 1; f.ww = g.wt * g.wh * g.ww;
+  Geo o = make_geo(f);
+  const long long frame = (long long)g.H * g.W;
+  const long long ns = (frame + o.blk - 1) / o.blk;
+  o.nsink = (int)(ns < o.Nb ? ns : o.Nb);
   return o;
 }
 

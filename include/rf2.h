@@ -66,7 +66,16 @@ enum rf2_flags {
      * [B, Npad, heads, D].  The kernels then gather each 3D window straight from model
      * order (pad tokens read as zeros) and write O rows to their tokens; the results are
      * those of the window-order call on rf2_permute'd inputs, bit for bit. */
-    RF2_RASTER = 4u
+    RF2_RASTER = 4u,
+    /* The "without 3D permutation" ablation (sciencestack page, Figure 3 (b)): a block is
+     * blk = wt*wh*ww consecutive tokens of model (raster) order instead of a 3D window.
+     * Every entry point that takes flags then works on the flat geometry T' = H' = 1,
+     * W' = N with window (1, 1, blk): Nb = ceil(N/blk), Npad = Nb*blk (the last block is
+     * padded at its end), and "window order" is model order padded to Npad rows.  The
+     * first-frame sink becomes the blocks that hold a token of frame 0, the first
+     * ceil(H*W/blk) blocks.  rf2_permute and rf2_unpermute take no flags and keep
+     * the 3D windows. */
+    RF2_NO_PERMUTE = 8u
 };
 
 /* rf2_permute - 3D window permutation (mlsanity index page, Abstract, insight (2)
@@ -86,7 +95,7 @@ int rf2_unpermute(const void* xp, void* x, const rf2_geom* g, void* stream);
 /* rf2_kept_count - number of key blocks every (b, head, query block) row keeps
  * (sciencestack page, TL;DR: target sparsity; mlsanity index page, insight (3): the
  * first-frame sink).  The sink S is the Hp/wh * Wp/ww blocks of temporal window 0 when
- * `sink` is non-zero.  Returns the count (>= 1) or -RF2_ERR_* on a bad argument.
+ * `sink` is non-zero (with RF2_NO_PERMUTE: the ceil(H*W/blk) blocks that hold frame 0).  Returns the count (>= 1) or -RF2_ERR_* on a bad argument.
  * This is the minimum `kmax` of rf2_predict_mask. */
 int rf2_kept_count(const rf2_geom* g, double sparsity, int sink, unsigned flags);
 

@@ -35,6 +35,8 @@ Parity status of each function (what pins it, in tests/test_oracle.py):
   sparse_attention                       : dense brute force at 0% sparsity, torch SDPA (fp64),
                                            explicit -inf masked dense attention, closed forms
   schedule_action                        : hand-worked step tables (tests/golden/schedule_actions.txt)
+  no_permute geometry (raster blocks)    : hand-worked positions and sink, equality with the
+                                           (T, 1, W) grid cut into (1, 1, blk) windows
 The end-to-end RF2 numbers themselves are not printed on the pages (no worked example),
 so the method's outputs beyond these pins are "parity unpinned by the pages".
 """
@@ -61,6 +63,9 @@ class Geom:
     wt: int
     wh: int
     ww: int
+    # "Without 3D permutation" ablation (sciencestack page, Figure 3 (b)): a block is blk
+    # consecutive tokens of the raster order instead of a 3D window.
+    no_permute: bool = False
 
     @property
     def N(self) -> int:
@@ -96,6 +101,8 @@ class Geom:
 
     @property
     def Nb(self) -> int:
+        if self.no_permute:
+            return -(-self.N // self.blk)
         return self.nbt * self.nbh * self.nbw
 
     @property
@@ -113,7 +120,12 @@ def window_positions(g: Geom) -> np.ndarray:
     RF2 abstract, insight (2) / TL;DR "3D window permutation": token (t, h, w) belongs to
     window (t//wt, h//wh, w//ww); windows are numbered row-major over the padded grid and
     tokens inside a window row-major over (t%wt, h%wh, w%ww).
+
+    no_permute: the sequence stays in raster order (Figure 3 (b)), so token n sits at
+    position n and block n // blk holds it.
     """
+    if g.no_permute:
+        return np.arange(g.N).reshape(g.T, g.H, g.W)
     t = np.arange(g.T)[:, None, None]
     h = np.arange(g.H)[None, :, None]
     w = np.arange(g.W)[None, None, :]
@@ -127,6 +139,11 @@ def position_to_token(g: Geom) -> np.ndarray:
     """Inverse map, built independently of window_positions: for every permuted position
     p in [0, Npad), the raster token index (t*H + h)*W + w, or -1 for a pad position."""
     out = np.full(g.Npad, -1, dtype=np.int64)
+    if g.no_permute:
+        # raster blocks: position p holds token p; the tail of the last block is padding
+        out[:g.N] = np.arange(g.N)
+        out.setflags(write=False)
+        return out
     for p in range(g.Npad):
         block, offset = divmod(p, g.blk)
         tb, rest = divmod(block, g.nbh * g.nbw)
@@ -170,7 +187,12 @@ def block_valid_counts(g: Geom) -> np.ndarray:
 def sink_blocks(g: Geom) -> np.ndarray:
     """Block ids of the first-frame sink: every window whose temporal index is 0 (RF2
     abstract, insight (3) 'first-frame sink').  With wt > 1 these windows hold frames
-    0..wt-1; a block is kept or dropped as a whole."""
+    0..wt-1; a block is kept or dropped as a whole.
+
+    no_permute: the blocks that hold at least one token of frame 0, i.e. those starting
+    before token H*W of the raster order."""
+    if g.no_permute:
+        return np.array([j for j in range(g.Nb) if j * g.blk < g.H * g.W], dtype=np.int64)
     return np.arange(g.nbh * g.nbw)
 
 

@@ -150,3 +150,31 @@ def test_schedule_action_matches_oracle_and_rejects_bad_input():
         assert lib.rf2_schedule_action(ctypes.byref(bad), 0) == -_lib.RF2_ERR_INVALID_ARG
     assert lib.rf2_schedule_action(None, 0) == -_lib.RF2_ERR_INVALID_ARG
     assert rf2.Schedule(50, 0.1, 5).action(5) == _lib.RF2_STEP_PREDICT
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_no_permute_kept_count_and_workspace_match_oracle(name):
+    """RF2_NO_PERMUTE: the library's flat geometry (blocks of consecutive raster tokens,
+    sink = blocks holding frame 0) agrees with the oracle's own restatement."""
+    wl = WORKLOADS[name]
+    g = rf2.Geometry(**wl.geom(), no_permute=True)
+    og = O.geom(**wl.geom(), no_permute=True)
+    assert (g.Nb, g.Npad) == (og.Nb, og.Npad)
+    for i in range(0, 101, 5):
+        s = i / 100
+        for sink in (False, True):
+            for additive in (False, True):
+                assert rf2.kept_count(g, s, sink, additive) == O.kept_count(og, s, sink, additive), (s, sink, additive)
+    ws_mask = rf2.workspace_size(g, 0.8, True, attention=False)
+    assert ws_mask >= 2 * 3 * g.B * g.heads * g.Nb * g.D * 2 + g.B * g.heads * g.Nb * g.Nb * 4
+    ws_w = rf2.workspace_size(rf2.Geometry(**wl.geom()), 0.8, True, attention=False)
+    assert (ws_mask < ws_w) == (g.Nb < rf2.Geometry(**wl.geom()).Nb)
+
+
+def test_no_permute_geometry_has_no_window_permutation():
+    g = _g(no_permute=True)
+    x = __import__("torch").zeros((g.B, g.N, g.heads, g.D))
+    with pytest.raises(ValueError):
+        rf2.permute(x, g)
+    with pytest.raises(ValueError):
+        rf2.unpermute(x, g)

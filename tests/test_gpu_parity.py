@@ -376,3 +376,79 @@ def test_step_attention_follows_its_schedule():
         assert torch.equal(idx, i1) and torch.equal(cnt, c1)   # the lists of that layer's predict step
     with pytest.raises(RuntimeError):
         rf2.StepAttention(g, 0.5, wl.sink, schedule=sched)(0, 2, *inputs[0, 2])               # reuse before predict
+
+
+# ----------------------------------------------------------------------------- no-permute ablation
+
+NO_PERMUTE = [
+    dict(B=2, heads=2, T=3, H=10, W=13, D=64, wt=1, wh=8, ww=8),     # 7 blocks of 64, tail of 6
+    dict(B=1, heads=2, T=5, H=9, W=17, D=128, wt=2, wh=8, ww=8),     # 6 blocks of 128, tail of 125
+    dict(B=1, heads=3, T=2, H=16, W=16, D=128, wt=1, wh=8, ww=16),   # frames are whole blocks
+]
+
+
+@pytest.mark.parametrize("shape", NO_PERMUTE)
+def test_no_permute_mask_and_attention_ragged(shape):
+    """RF2_NO_PERMUTE (raster blocks): kept lists bit-exact outside the near-cut window,
+    attention within tolerance, model-order and padded-order calls bit-identical."""
+    g = rf2.Geometry(**shape, no_permute=True)
+    og = O.geom(**shape, no_permute=True)
+    q, k, v = _rand_bits(g, 1300)
+    qp, kp, vp = (O.permute(a, og) for a in (q, k, v))          # raster order, tail padded
+    qf, kf, vf = (bf16_bits_to_f64(a) for a in (qp, kp, vp))
+    for s, sink, additive in ((0.5, True, False), (0.5, True, True), (0.7, False, False)):
+        sel = O.predict_mask(qf, kf, og, s, sink, additive)
+        idx_r, cnt_r = rf2.predict_mask(to_dev(q), to_dev(k), g, s, sink, additive, checked=True, raster=True)
+        compare_lists(idx_r.cpu().numpy(), cnt_r.cpu().numpy(), sel)
+        idx_w, cnt_w = rf2.predict_mask(to_dev(qp), to_dev(kp), g, s, sink, additive, checked=True)
+        assert torch.equal(idx_r, idx_w) and torch.equal(cnt_r, cnt_w)
+    sel = O.predict_mask(qf, kf, og, 0.5, True)
+    idx = torch.from_numpy(sel.idx).cuda()
+    cnt = torch.full(sel.idx.shape[:3], sel.kept, dtype=torch.int32, device="cuda")
+    o_r = rf2.sparse_attn(to_dev(q), to_dev(k), to_dev(v), idx, cnt, g, checked=True, raster=True)
+    o_w = rf2.sparse_attn(to_dev(qp), to_dev(kp), to_dev(vp), idx, cnt, g, checked=True)
+    assert torch.equal(o_r.view(torch.int16), o_w[:, :og.N].contiguous().view(torch.int16))
+    got = to_f64(o_r)
+    sc = 1 / np.sqrt(og.D)
+    ref = np.zeros_like(got)
+    for b in range(og.B):
+        for h in range(og.heads):
+            for i in range(og.Nb):
+                rows = O.attention_block(qf, kf, vf, og, b, h, i, sel.idx[b, h, i], sc)
+                lo, hi = i * og.blk, min((i + 1) * og.blk, og.N)
+                ref[b, lo:hi, h] = rows[:hi - lo]
+    print(shape, assert_close(got, ref, "no_permute sparse_attn"))
+    out, gidx = rf2.attention(to_dev(q), to_dev(k), to_dev(v), g, 0.5, True, return_idx=True, checked=True)
+    compare_lists(gidx.cpu().numpy(), cnt.cpu().numpy(), sel)
+    ref_e2e, _ = O.attention(bf16_bits_to_f64(q), bf16_bits_to_f64(k), bf16_bits_to_f64(v), og, 0.5, True)
+    if torch.equal(gidx.cpu(), torch.from_numpy(sel.idx)):
+        assert_close(to_f64(out), ref_e2e, "no_permute attention")
+
+
+def test_no_permute_wan720p_end_to_end_sampled():
+    """The ablation at the 720p video shape: 591 raster blocks of 128 tokens (last one
+    80 tokens), 29 sink blocks, 119 kept per row at 80 % sparsity."""
+    wl = WORKLOADS["wan720p"]
+    g = rf2.Geometry(**wl.geom(), no_permute=True)
+    og = O.geom(**wl.geom(), no_permute=True)
+    q, k, v = _inputs("wan720p")
+    out, idx = rf2.attention(to_dev(q), to_dev(k), to_dev(v), g, wl.sparsity, wl.sink,
+                             return_idx=True, checked=True)
+    qf, kf, vf = (bf16_bits_to_f64(O.permute(a, og)) for a in (q, k, v))
+    sel = O.predict_mask(qf, kf, og, wl.sparsity, wl.sink)
+    assert sel.kept == 119 and og.Nb == 591
+    gidx = idx.cpu().numpy()
+    stats = compare_lists(gidx, np.full(gidx.shape[:3], sel.kept), sel)
+    got = to_f64(out)
+    rng = np.random.default_rng(11)
+    picks = {(int(rng.integers(og.heads)), int(rng.integers(og.Nb))) for _ in range(10)}
+    picks |= {(0, 0), (og.heads - 1, og.Nb - 1), (3, 28)}     # first, ragged last, last sink block
+    got_rows, ref_rows = [], []
+    for h, i in sorted(picks):
+        if not np.array_equal(gidx[0, h, i], sel.idx[0, h, i]):
+            continue
+        rows = O.attention_block(qf, kf, vf, og, 0, h, i, sel.idx[0, h, i], 1 / np.sqrt(og.D))
+        lo, hi = i * og.blk, min((i + 1) * og.blk, og.N)
+        ref_rows.append(rows[:hi - lo])
+        got_rows.append(got[0, lo:hi, h])
+    print("wan720p no_permute", stats, assert_close(np.concatenate(got_rows), np.concatenate(ref_rows), "wan720p"))

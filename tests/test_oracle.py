@@ -340,3 +340,69 @@ def test_schedule_invariants():
                 if n_dense < total:
                     assert acts[n_dense] == O.PREDICT                     # a mask exists before reuse
                 assert (O.REUSE in acts) == (interval > 1 and total - n_dense > 1)
+
+
+# ----------------------------------------------------------------------------- no-permute ablation
+
+def _np_g(T, H, W, wt, wh, ww, B=1, heads=1, D=8):
+    return O.geom(B=B, heads=heads, T=T, H=H, W=W, D=D, wt=wt, wh=wh, ww=ww, no_permute=True)
+
+
+def test_no_permute_matches_hand_worked_table():
+    for ln in _golden_lines("no_permute_small.txt"):
+        lhs, rhs = ln.split(":")
+        f = lhs.split()
+        T, H, W, wt, wh, ww = map(int, f[:6])
+        s = float(f[6])
+        Nb, Npad, last, ns, kin, kadd = map(int, rhs.split())
+        g = _np_g(T, H, W, wt, wh, ww)
+        assert (g.Nb, g.Npad) == (Nb, Npad)
+        cnt = O.block_valid_counts(g)
+        assert list(cnt[:-1]) == [g.blk] * (Nb - 1) and cnt[-1] == last
+        assert list(O.sink_blocks(g)) == list(range(ns))
+        assert O.kept_count(g, s, True) == kin
+        assert O.kept_count(g, s, True, sink_additive=True) == kadd
+
+
+def test_no_permute_keeps_raster_order_and_pads_the_tail():
+    g = _np_g(2, 3, 5, 1, 2, 4, heads=2, D=3)
+    # entries encode (b, token, head, d): the permuted tensor must hold token p at row p
+    x = np.arange(1 * g.N * 2 * 3, dtype=np.float64).reshape(1, g.N, 2, 3) + 1.0
+    xp = O.permute(x, g)
+    assert xp.shape == (1, 32, 2, 3)
+    np.testing.assert_array_equal(xp[:, :g.N], x)
+    assert np.all(xp[:, g.N:] == 0)
+    np.testing.assert_array_equal(O.unpermute(xp, g), x)
+    assert list(O.position_to_token(g)[28:]) == [28, 29, -1, -1]
+
+
+@pytest.mark.parametrize("T,H,W,blk", [(3, 4, 32, 64), (2, 8, 16, 128), (4, 2, 32, 64)])
+def test_no_permute_equals_flat_grid_cut_into_one_row_windows(T, H, W, blk):
+    """When a frame is a whole number of blocks, raster blocks are exactly the windows
+    (1, 1, blk) of the grid (T, 1, H*W), whose sink (temporal window 0) is frame 0: the
+    two geometries must give the same positions, sink, kept lists and outputs."""
+    g_np = O.geom(B=1, heads=2, T=T, H=H, W=W, D=16, wt=1, wh=1, ww=blk, no_permute=True)
+    g_w = O.geom(B=1, heads=2, T=T, H=1, W=H * W, D=16, wt=1, wh=1, ww=blk)
+    assert (g_np.Nb, g_np.Npad) == (g_w.Nb, g_w.Npad)
+    np.testing.assert_array_equal(O.window_positions(g_np).reshape(-1), O.window_positions(g_w).reshape(-1))
+    np.testing.assert_array_equal(O.position_to_token(g_np), O.position_to_token(g_w))
+    np.testing.assert_array_equal(O.sink_blocks(g_np), O.sink_blocks(g_w))
+    rng = np.random.default_rng(T * 100 + W)
+    q, k, v = (rng.standard_normal((1, T * H * W, 2, 16)) for _ in range(3))
+    for s in (0.5, 0.8):
+        a, sa = O.attention(q, k, v, g_np, s, True)
+        b, sb = O.attention(q, k, v, g_w, s, True)
+        np.testing.assert_array_equal(sa.idx, sb.idx)
+        np.testing.assert_array_equal(a, b)
+
+
+def test_no_permute_ragged_tail_is_masked():
+    """A partial last block: its pad keys carry no weight (the tail query rows match
+    dense attention restricted to the kept real tokens)."""
+    g = O.geom(B=1, heads=1, T=3, H=10, W=13, D=8, wt=1, wh=8, ww=8, no_permute=True)
+    rng = np.random.default_rng(3)
+    q, k, v = (rng.standard_normal((1, g.N, 1, 8)) for _ in range(3))
+    out, sel = O.attention(q, k, v, g, 0.0, True)
+    ref = O.dense_attention(q, k, v, 1 / math.sqrt(8))
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    assert sel.kept == g.Nb == 7

@@ -82,3 +82,19 @@ def test_noalloc_model_order_matches_window_order():
         idx, cnt = _noalloc(qd, kd, g, wl.sparsity, wl.sink, _lib.RF2_RASTER, kept)
         torch.cuda.synchronize()
         assert torch.equal(idx, ref_idx) and torch.equal(cnt, ref_cnt)
+
+
+def test_noalloc_no_permute_matches_predict_mask():
+    """RF2_NO_PERMUTE (raster blocks) through the no-allocation call: the same lists as
+    rf2_predict_mask with the same flags."""
+    wl = WORKLOADS["video480p"]
+    g = rf2.Geometry(**wl.geom(), no_permute=True)
+    q, k, _ = gen_qkv(wl)
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+    qd, kd = to_dev(q), to_dev(k)
+    kept = rf2.kept_count(g, wl.sparsity, wl.sink)
+    ref_idx, ref_cnt = rf2.predict_mask(qd, kd, g, wl.sparsity, wl.sink, kmax=kept, raster=True)
+    idx, cnt = _noalloc(qd, kd, g, wl.sparsity, wl.sink, _lib.RF2_RASTER | _lib.RF2_NO_PERMUTE, kept)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, ref_idx) and torch.equal(cnt, ref_cnt)
+    assert int(cnt[0, 0, 0]) == kept
