@@ -35,6 +35,7 @@ __all__ = [
     "gen_tensor",
     "gen_qkv",
     "gen_tensor_torch",
+    "gen_pattern_heads",
     "bf16_bits_to_f64",
     "f32_to_bf16_bits",
 ]
@@ -184,3 +185,38 @@ def gen_tensor_torch(B: int, T: int, H: int, W: int, heads: int, D: int, seed: i
             x.add_(torch.bmm(pa, qw).permute(1, 2, 0))
             out[b, t] = x.to(torch.bfloat16)
     return out.view(B, T * H * W, heads, D)
+
+
+def gen_pattern_heads(B: int, T: int, H: int, W: int, heads: int, D: int, seed: int,
+                      kinds: str, amp: float = 2.0, noise: float = 0.3) -> Sequence[np.ndarray]:
+    """Q, K, V raw bf16 bits [B, T*H*W, heads, D] whose heads follow planted attention
+    patterns, one letter per head in `kinds`:
+
+      't' - Q = K = amp * u[h, w] + noise * eps: one random vector per spatial position,
+            the same in every frame (each token matches its own location in all frames);
+      's' - Q = K = amp * v[t] + noise * eps: one random vector per frame (each token
+            matches every token of its own frame);
+      'x' - Q, K = eps: unstructured.
+    u, v, eps ~ N(0, 1) from numpy's PCG64(seed); V = eps for every head.  Rounded to
+    bf16 (nearest even)."""
+    assert len(kinds) == heads
+    rng = np.random.Generator(np.random.PCG64(seed))
+    N = T * H * W
+    q = np.empty((B, N, heads, D), dtype=np.float32)
+    k = np.empty_like(q)
+    for b in range(B):
+        for h, kind in enumerate(kinds):
+            if kind == "t":
+                base = np.tile(rng.standard_normal((H * W, D)), (T, 1)) * amp
+            elif kind == "s":
+                base = np.repeat(rng.standard_normal((T, D)), H * W, axis=0) * amp
+            else:
+                base = None
+            if base is None:
+                q[b, :, h] = rng.standard_normal((N, D))
+                k[b, :, h] = rng.standard_normal((N, D))
+            else:
+                q[b, :, h] = base + noise * rng.standard_normal((N, D))
+                k[b, :, h] = base + noise * rng.standard_normal((N, D))
+    v = rng.standard_normal((B, N, heads, D)).astype(np.float32)
+    return [f32_to_bf16_bits(a) for a in (q, k, v)]
