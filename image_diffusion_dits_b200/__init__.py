@@ -21,7 +21,8 @@ from ._lib import RF2_CHECKED, RF2_SINK_ADDITIVE, Rf2Geom
 
 __all__ = [
     "Geometry", "Rf2Error", "permute", "unpermute", "kept_count", "workspace_size",
-    "predict_mask", "sparse_attn", "attention", "library",
+    "predict_mask", "sparse_attn", "attention", "library", "Schedule", "StepAttention",
+    "V1Params", "v1_kmax", "v1_workspace_size", "v1_predict_mask",
 ]
 
 
@@ -281,6 +282,67 @@ class StepAttention:
         elif layer not in self._lists:
             raise RuntimeError(f"step {step} reuses the mask of layer {layer!r}, which has none predicted yet")
         return sparse_attn(q, k, v, *self._lists[layer], g, out=out, raster=True)
+
+
+@dataclasses.dataclass(frozen=True)
+class V1Params:
+    """Parameters of the RainFusion v1 mask generators (rf2_v1_params): band half-width as
+    a fraction of the axis, checkerboard stride of textural heads, recall threshold of
+    the head classification, global sampling interval (0: T), RainFusion+ dynamic
+    bandwidth and its recall target."""
+
+    bandwidth: float = 0.25
+    tau: int = 2
+    alpha: float = 0.9
+    omega: int = 0
+    dynamic: bool = False
+    recall_target: float = 0.9
+
+    def c(self) -> _lib.Rf2V1Params:
+        return _lib.Rf2V1Params(float(self.bandwidth), int(self.tau), float(self.alpha), int(self.omega),
+                                int(bool(self.dynamic)), float(self.recall_target))
+
+
+def v1_kmax(g: Geometry, params: V1Params = V1Params()) -> int:
+    cg, cp = g.c(), params.c()
+    k = library().rf2_v1_kmax(ctypes.byref(cg), ctypes.byref(cp), g.flags)
+    if k < 0:
+        raise Rf2Error(-k, "rf2_v1_kmax")
+    return k
+
+
+def v1_workspace_size(g: Geometry, params: V1Params = V1Params()) -> int:
+    cg, cp = g.c(), params.c()
+    n = library().rf2_v1_workspace_size(ctypes.byref(cg), ctypes.byref(cp), g.flags)
+    if n == 0:
+        raise Rf2Error(_lib.RF2_ERR_INVALID_ARG, "rf2_v1_workspace_size")
+    return n
+
+
+def v1_predict_mask(q: torch.Tensor, k: torch.Tensor, g: Geometry, params: V1Params = V1Params(),
+                    kmax: Optional[int] = None, checked: bool = False, ws: Optional[torch.Tensor] = None):
+    """RainFusion v1 kept lists from model-order q, k [B, N, heads, D]: ARM classifies every
+    head (temporal / spatial / textural) from its sampled recall and the lists follow the
+    class's block mask.  Returns (idx [B, heads, Nb, kmax], cnt [B, heads, Nb],
+    head_class [B, heads], recall [B, heads, 2, 4]); feed idx, cnt to sparse_attn(...,
+    raster=True)."""
+    for t, n in ((q, "q"), (k, "k")):
+        _cuda_bf16(t, n, (g.B, g.N, g.heads, g.D))
+    kk = v1_kmax(g, params) if kmax is None else kmax
+    dev = q.device
+    idx = torch.empty((g.B, g.heads, g.Nb, kk), dtype=torch.int32, device=dev)
+    cnt = torch.empty((g.B, g.heads, g.Nb), dtype=torch.int32, device=dev)
+    cls = torch.empty((g.B, g.heads), dtype=torch.int32, device=dev)
+    rec = torch.empty((g.B, g.heads, 2, 4), dtype=torch.float32, device=dev)
+    nbytes = v1_workspace_size(g, params)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    cg, cp = g.c(), params.c()
+    _check(library().rf2_v1_predict_mask(q.data_ptr(), k.data_ptr(), ctypes.byref(cg), ctypes.byref(cp),
+                                         _flags(g, False, checked), idx.data_ptr(), cnt.data_ptr(), kk,
+                                         cls.data_ptr(), rec.data_ptr(), ws.data_ptr(), ws.numel(), _stream(q)),
+           "rf2_v1_predict_mask")
+    return idx, cnt, cls, rec
 
 
 def default_scale(D: int) -> float:

@@ -33,8 +33,15 @@ EXPORTS = (
     "rf2_sparse_attn",
     "rf2_attention",
     "rf2_schedule_action",
+    "rf2_v1_kmax",
+    "rf2_v1_workspace_size",
+    "rf2_v1_predict_mask",
     "rf2_status_string",
 )
+
+RF2_V1_TEMPORAL = 0
+RF2_V1_SPATIAL = 1
+RF2_V1_TEXTURAL = 2
 
 
 RF2_STEP_DENSE = 0
@@ -45,6 +52,11 @@ RF2_STEP_REUSE = 2
 class Rf2Schedule(ctypes.Structure):
     _fields_ = [("total_steps", ctypes.c_int), ("dense_fraction", ctypes.c_double),
                 ("predict_interval", ctypes.c_int)]
+
+
+class Rf2V1Params(ctypes.Structure):
+    _fields_ = [("bandwidth", ctypes.c_double), ("tau", ctypes.c_int), ("alpha", ctypes.c_double),
+                ("omega", ctypes.c_int), ("dynamic", ctypes.c_int), ("recall_target", ctypes.c_double)]
 
 
 class Rf2Geom(ctypes.Structure):
@@ -70,6 +82,10 @@ _SIGS = {
     "rf2_attention": (ctypes.c_int, [_vp, _vp, _vp, _gp, ctypes.c_double, ctypes.c_int, ctypes.c_float,
                                      _vp, _i32p, _vp, ctypes.c_size_t, ctypes.c_uint, _vp]),
     "rf2_schedule_action": (ctypes.c_int, [ctypes.POINTER(Rf2Schedule), ctypes.c_int]),
+    "rf2_v1_kmax": (ctypes.c_int, [_gp, ctypes.POINTER(Rf2V1Params), ctypes.c_uint]),
+    "rf2_v1_workspace_size": (ctypes.c_size_t, [_gp, ctypes.POINTER(Rf2V1Params), ctypes.c_uint]),
+    "rf2_v1_predict_mask": (ctypes.c_int, [_vp, _vp, _gp, ctypes.POINTER(Rf2V1Params), ctypes.c_uint, _i32p,
+                                           _i32p, ctypes.c_int, _i32p, _vp, _vp, ctypes.c_size_t, _vp]),
     "rf2_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
 

@@ -116,9 +116,107 @@ int finish_checked(unsigned flags, const int32_t* status_dev, cudaStream_t s) {
   return st;
 }
 
+// RainFusion v1 generators: validated arguments, kernel arguments and kmax.
+struct V1Call {
+  Geo geo;
+  rf2::Rf1Args a;
+  int kmax;
+};
+
+int v1_radius(double bw, int C) { return (int)floor(bw * (double)C + 1e-6); }
+
+int v1_prepare(const rf2_geom* g, const rf2_v1_params* p, unsigned flags, V1Call* c) {
+  int st = check_geom(g, 0);
+  if (st != RF2_OK) return st;
+  if (flags & RF2_NO_PERMUTE) return RF2_ERR_UNSUPPORTED;
+  if (p == nullptr || !(p->bandwidth > 0.0 && p->bandwidth <= 1.0) || p->tau < 1 ||
+      !(p->alpha >= 0.0 && p->alpha <= 1.0) || !(p->recall_target >= 0.0 && p->recall_target <= 1.0) ||
+      p->omega < 0 || (p->dynamic != 0 && p->dynamic != 1))
+    return RF2_ERR_INVALID_ARG;
+  Geo geo = rf2::make_geo(*g);
+  if ((long long)geo.B * geo.heads > 65535) return RF2_ERR_UNSUPPORTED;  // grid z
+  rf2::Rf1Args a;
+  const long long omega = p->omega == 0 ? g->T : p->omega;
+  a.S[0] = g->H * g->W;
+  a.S[1] = (int)((geo.N + omega - 1) / omega);
+  a.coord_off[0] = 0;
+  a.coord_off[1] = a.S[0];
+  a.tiles_max = (max(a.S[0], a.S[1]) + 127) / 128;
+  a.omega = (int)omega;
+  a.HW = g->H * g->W;
+  a.W = g->W; a.wh = g->wh; a.ww = g->ww; a.nbw = geo.nbw; a.wt = g->wt; a.heads = g->heads;
+  const double levels[4] = {p->bandwidth, 0.125, 0.25, 0.5};
+  const int P = geo.nbh * geo.nbw;
+  for (int l = 0; l < 4; ++l) {
+    a.R[0][l] = v1_radius(levels[l], P);
+    a.R[1][l] = v1_radius(levels[l], geo.nbt);
+  }
+  a.tau = p->tau;
+  a.dynamic = p->dynamic;
+  a.alpha = (float)p->alpha;
+  a.target = (float)p->recall_target;
+  a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)g->D));
+  // longest list: temporal nbt * min(P, 2R+1), spatial min(nbt, 2R+1) * P, textural
+  // nbt * (windows of a slab on the checkerboard)
+  int kmax = 0;
+  for (int l = 0; l < (p->dynamic ? 4 : 1); ++l) {
+    kmax = max(kmax, geo.nbt * min(P, 2 * a.R[0][l] + 1));
+    kmax = max(kmax, min(geo.nbt, 2 * a.R[1][l] + 1) * P);
+  }
+  int tex = 0;
+  for (int sw = 0; sw < P; ++sw) tex += ((sw / geo.nbw + sw % geo.nbw) % p->tau) == 0;
+  kmax = max(kmax, geo.nbt * tex);
+  c->geo = geo;
+  c->a = a;
+  c->kmax = kmax;
+  return RF2_OK;
+}
+
+size_t v1_ws_bytes(const V1Call& c) {
+  return kAlign + align_up(rf2::rf1_scratch_layout(c.geo, c.a, nullptr).bytes);
+}
+
 }  // namespace
 
 extern "C" {
+
+int rf2_v1_kmax(const rf2_geom* g, const rf2_v1_params* p, unsigned flags) {
+  V1Call c;
+  int st = v1_prepare(g, p, flags, &c);
+  return st != RF2_OK ? -st : c.kmax;
+}
+
+size_t rf2_v1_workspace_size(const rf2_geom* g, const rf2_v1_params* p, unsigned flags) {
+  V1Call c;
+  if (v1_prepare(g, p, flags, &c) != RF2_OK) return 0;
+  return v1_ws_bytes(c);
+}
+
+int rf2_v1_predict_mask(const void* q, const void* k, const rf2_geom* g, const rf2_v1_params* p,
+                        unsigned flags, int32_t* idx, int32_t* cnt, int kmax, int32_t* head_class,
+                        float* recall, void* ws, size_t ws_bytes, void* stream) {
+  V1Call c;
+  int st = v1_prepare(g, p, flags, &c);
+  if (st != RF2_OK) return st;
+  if (q == nullptr || k == nullptr || idx == nullptr || cnt == nullptr) return RF2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || ((uintptr_t)idx & 3u) || ((uintptr_t)cnt & 3u) ||
+      ((uintptr_t)head_class & 3u) || ((uintptr_t)recall & 3u))
+    return RF2_ERR_ALIGNMENT;
+  if (kmax < c.kmax) return RF2_ERR_INVALID_ARG;
+  if (ws == nullptr) return RF2_ERR_WORKSPACE;
+  if (!aligned16(ws)) return RF2_ERR_ALIGNMENT;
+  if (ws_bytes < v1_ws_bytes(c)) return RF2_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int32_t* status = reinterpret_cast<int32_t*>(base);
+  const rf2::Rf1Scratch w = rf2::rf1_scratch_layout(c.geo, c.a, base + kAlign);
+  cudaStream_t s = (cudaStream_t)stream;
+  log_geo("v1_predict_mask", c.geo, c.kmax);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), s);
+  if (e == cudaSuccess) e = rf2::launch_rf1(q, k, c.geo, c.a, w, head_class, recall, idx, cnt, kmax, status, s);
+  if (e != cudaSuccess) return RF2_ERR_CUDA;
+  return finish_checked(flags, status, s);
+}
+
 
 const char* rf2_status_string(int status) {
   switch (status) {

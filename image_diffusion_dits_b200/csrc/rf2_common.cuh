@@ -118,6 +118,42 @@ inline MaskScratch mask_scratch_layout(const Geo& g, unsigned char* base) {
   return m;
 }
 
+// Arguments of the RainFusion v1 generators (host-derived, passed by value).  Sample p = 0
+// is the local sample (the H*W frame-0 tokens), p = 1 the global one (every omega-th
+// raster token).  R[p][l] is the band radius of level l = (static bandwidth, 1/8, 1/4,
+// 1/2) on that sample's axis (windows of a slab for p = 0, temporal blocks for p = 1).
+struct Rf1Args {
+  int S[2];           // samples
+  int coord_off[2];   // offsets of each sample's coordinates in the coordinate table
+  int tiles_max;      // max over p of ceil(S[p] / 128)
+  int omega, HW, W, wh, ww, nbw, wt, heads;
+  int R[2][4];
+  int tau, dynamic;
+  float alpha, target, scale_log2;
+};
+
+// Scratch of the v1 generators (after the call's status word).
+struct Rf1Scratch {
+  int* coords;       // [S0 + S1] window coordinate of every sampled token
+  float* partial;    // [B*heads][2][tiles_max][4 warps][4 levels]
+  int* clsparam;     // [B*heads][2]: class, radius or stride
+  size_t bytes;
+};
+
+inline Rf1Scratch rf1_scratch_layout(const Geo& g, const Rf1Args& a, unsigned char* base) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  Rf1Scratch w;
+  size_t off = 0;
+  w.coords = reinterpret_cast<int*>(base + off);
+  off += up((size_t)(a.S[0] + a.S[1]) * sizeof(int));
+  w.partial = reinterpret_cast<float*>(base + off);
+  off += up((size_t)g.B * g.heads * 2 * a.tiles_max * 16 * sizeof(float));
+  w.clsparam = reinterpret_cast<int*>(base + off);
+  off += up((size_t)g.B * g.heads * 2 * sizeof(int));
+  w.bytes = off;
+  return w;
+}
+
 // cuTensorMapEncodeTiled from the driver (looked up once), or null if unavailable.
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -149,5 +185,11 @@ cudaError_t launch_topk(const float* scores, int32_t* idx, int32_t* cnt, int kma
 cudaError_t launch_sparse_attn(const void* qp, const void* kp, const void* vp,
                                const int32_t* idx, const int32_t* cnt, int kmax, const Geo& g,
                                float scale, void* op, int32_t* status, bool raster, cudaStream_t s);
+
+// RainFusion v1: ARM recall of the two samples, head classes, kept lists.  q, k in model
+// order [B, N, heads, D].  cls_out [B*heads] and recall_out [B*heads][2][4] may be null.
+cudaError_t launch_rf1(const void* q, const void* k, const Geo& g, const Rf1Args& a, const Rf1Scratch& w,
+                       int32_t* cls_out, float* recall_out, int32_t* idx, int32_t* cnt, int kmax,
+                       int32_t* status, cudaStream_t s);
 
 }  // namespace rf2

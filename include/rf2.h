@@ -212,6 +212,62 @@ enum rf2_step_action {
  * -RF2_ERR_INVALID_ARG on a bad schedule or a step outside [0, total_steps). */
 int rf2_schedule_action(const rf2_schedule* schedule, int step);
 
+/* RainFusion (v1) mask generators (pith.science review of "RainFusion: Adaptive Video
+ * Generation Acceleration via Multi-Dimensional Visual Redundancy": "What carries the
+ * argument", "Core claim", "Free parameters").  They emit kept lists for the same
+ * block-sparse attention (rf2_sparse_attn with RF2_RASTER).  Blocks are the 3D windows of
+ * rf2_geom; a block's coordinates are its temporal block tb and its window index
+ * sw = hb * nbw + wb inside a temporal slab (nbw = Wp/ww, P = nbh * nbw windows per slab).
+ * Head patterns, per (query block i, key block j):
+ *   temporal, radius R: |sw_i - sw_j| <= R     spatial, radius R: |tb_i - tb_j| <= R
+ *   textural, stride tau: (hb_j + wb_j) mod tau == 0 (a checkerboard of windows)
+ * with R = floor(b * C + 1e-6) for bandwidth b, C = P (temporal) or Tp/wt (spatial).
+ * ARM (adaptive recognition) recall of a band: mean over sampled query tokens of the
+ * softmax mass (over the sampled keys, scale 1/sqrt(D)) whose key lies in the band, the
+ * band judged on the windows of the two tokens.  Local sample: the H*W tokens of frame 0,
+ * scored with the temporal band; global sample: raster tokens 0, omega, 2 omega, ...,
+ * scored with the spatial band.  A head is temporal if its local recall at `bandwidth`
+ * reaches alpha, else spatial if its global recall does, else textural.  With `dynamic`
+ * (RainFusion+), a temporal or spatial head then takes the smallest bandwidth of 1/8,
+ * 1/4, 1/2 whose recall reaches recall_target (else 1/2). */
+typedef struct rf2_v1_params {
+    double bandwidth;      /* band half-width as a fraction of the axis, (0, 1]; pages: 1/4  */
+    int tau;               /* checkerboard stride of textural heads, >= 1; pages: 2          */
+    double alpha;          /* recall threshold of the classification, [0, 1]; not given: 0.9 */
+    int omega;             /* global sampling interval in tokens, >= 0; 0 means T            */
+    int dynamic;           /* 1: RainFusion+ bandwidth per head                              */
+    double recall_target;  /* RainFusion+ recall target, [0, 1]; pages: 0.9                  */
+} rf2_v1_params;
+
+/* Head classes written by rf2_v1_predict_mask. */
+enum rf2_v1_class { RF2_V1_TEMPORAL = 0, RF2_V1_SPATIAL = 1, RF2_V1_TEXTURAL = 2 };
+
+/* rf2_v1_kmax - the longest kept list any head class can produce for these parameters
+ * (the minimum kmax of rf2_v1_predict_mask), or -RF2_ERR_* on a bad argument.  flags:
+ * RF2_NO_PERMUTE is not supported (the patterns are defined on 3D windows). */
+int rf2_v1_kmax(const rf2_geom* g, const rf2_v1_params* p, unsigned flags);
+
+/* rf2_v1_workspace_size - device scratch of rf2_v1_predict_mask (status word, sample
+ * coordinates, per-warp recall sums, head classes); 0 on a bad argument. */
+size_t rf2_v1_workspace_size(const rf2_geom* g, const rf2_v1_params* p, unsigned flags);
+
+/* rf2_v1_predict_mask - ARM classification of every (b, head) and its kept lists, all on
+ * the device (no host synchronisation unless RF2_CHECKED).
+ *   q, k : [B, N, heads, D] bf16, model order (read).
+ *   idx  : [B, heads, Nb, kmax] int32 (written): ascending kept block ids, then -1.
+ *   cnt  : [B, heads, Nb] int32 (written): kept count of each row (rows of one head differ
+ *          at the band ends).
+ *   head_class : optional [B, heads] int32 rf2_v1_class (may be NULL).
+ *   recall     : optional [B, heads, 2, 4] float (may be NULL): local then global
+ *          sample, levels (bandwidth, 1/8, 1/4, 1/2).
+ *   kmax >= rf2_v1_kmax(...) else RF2_ERR_INVALID_ARG.
+ *   ws, ws_bytes : device scratch of at least rf2_v1_workspace_size(...) bytes.
+ * Errors: RF2_ERR_INVALID_ARG, RF2_ERR_UNSUPPORTED, RF2_ERR_ALIGNMENT, RF2_ERR_WORKSPACE,
+ *         RF2_ERR_CUDA, and (checked mode) RF2_ERR_TIMEOUT. */
+int rf2_v1_predict_mask(const void* q, const void* k, const rf2_geom* g, const rf2_v1_params* p,
+                        unsigned flags, int32_t* idx, int32_t* cnt, int kmax, int32_t* head_class,
+                        float* recall, void* ws, size_t ws_bytes, void* stream);
+
 /* rf2_status_string - static, human-readable text of a status code. */
 const char* rf2_status_string(int status);
 

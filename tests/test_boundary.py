@@ -178,3 +178,31 @@ def test_no_permute_geometry_has_no_window_permutation():
         rf2.permute(x, g)
     with pytest.raises(ValueError):
         rf2.unpermute(x, g)
+
+
+V1_GEOMS = [dict(B=1, heads=2, T=4, H=16, W=16, D=64, wt=1, wh=8, ww=8),
+            dict(B=2, heads=3, T=5, H=9, W=17, D=128, wt=2, wh=8, ww=8),
+            dict(B=1, heads=40, T=21, H=45, W=80, D=128, wt=2, wh=8, ww=8)]
+V1_PARAMS = [dict(), dict(dynamic=True), dict(bandwidth=0.5, tau=3), dict(bandwidth=0.125, tau=4, dynamic=True),
+             dict(bandwidth=1.0, tau=1)]
+
+
+@pytest.mark.parametrize("geo", V1_GEOMS)
+def test_v1_kmax_matches_oracle(geo):
+    g = rf2.Geometry(**geo)
+    og = O.geom(**geo)
+    for prm in V1_PARAMS:
+        assert rf2.v1_kmax(g, rf2.V1Params(**prm)) == O.rf1.rf1_kmax(og, O.rf1.Rf1Params(**prm)), prm
+        assert rf2.v1_workspace_size(g, rf2.V1Params(**prm)) > 0
+
+
+def test_v1_rejects_bad_parameters():
+    g = rf2.Geometry(**V1_GEOMS[0])
+    for bad in (dict(bandwidth=0.0), dict(bandwidth=1.5), dict(tau=0), dict(alpha=1.2), dict(omega=-1),
+                dict(recall_target=-0.1)):
+        with pytest.raises(rf2.Rf2Error) as ei:
+            rf2.v1_kmax(g, rf2.V1Params(**bad))
+        assert ei.value.code == _lib.RF2_ERR_INVALID_ARG, bad
+    with pytest.raises(rf2.Rf2Error) as ei:
+        rf2.v1_kmax(rf2.Geometry(**V1_GEOMS[0], no_permute=True))
+    assert ei.value.code == _lib.RF2_ERR_UNSUPPORTED
