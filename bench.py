@@ -45,6 +45,8 @@ def _args():
     p.add_argument("--sparsity", type=float, default=None)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-variants", action="store_true",
+                   help="skip the untimed-for-the-metric variant legs (no-permute ablation, RainFusion v1)")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--heads", type=int, default=None,
                    help="override the head count (smaller captures for profiling)")
@@ -194,6 +196,72 @@ def run_cpu_baseline(wl, sparsity, seconds, rows_cap=64):
     call_s = (per_row * og.Nb + t_mask_head) * og.heads * og.B
     return {"call_s": call_s, "cores": cores, "rows": done, "per_row_s": per_row,
             "mask_head_s": t_mask_head}
+
+
+def _time_legs(stream, iters, legs):
+    """Mean device time (ms) of each callable in `legs`, run in order per iteration, after
+    two warm-up iterations; CUDA events on the launching stream."""
+    import torch
+
+    for _ in range(2):
+        for f in legs:
+            f()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(legs) + 1)] for _ in range(iters)]
+    for it in range(iters):
+        ev[it][0].record(stream)
+        for j, f in enumerate(legs):
+            f()
+            ev[it][j + 1].record(stream)
+    torch.cuda.synchronize()
+    return [statistics.mean(ev[it][j].elapsed_time(ev[it][j + 1]) for it in range(iters)) for j in range(len(legs))]
+
+
+def run_variants(rf2, g, wl, sparsity, q, k, v, o, stream, dev, iters):
+    """Legs outside the headline step, on the same inputs: the "without 3D permutation"
+    ablation (blocks of consecutive raster tokens) and the RainFusion v1 generators (ARM
+    classification, RainFusion+) feeding the same attention kernel."""
+    import numpy as np
+    import torch
+
+    out = {}
+    gnp = rf2.Geometry(**wl.geom(), no_permute=True)
+    kept = rf2.kept_count(gnp, sparsity, wl.sink)
+    idx = torch.empty((g.B, g.heads, gnp.Nb, kept), dtype=torch.int32, device=dev)
+    cnt = torch.empty((g.B, g.heads, gnp.Nb), dtype=torch.int32, device=dev)
+    ws = torch.empty(rf2.workspace_size(gnp, sparsity, wl.sink, attention=False), dtype=torch.uint8, device=dev)
+    t_mask, t_attn = _time_legs(stream, iters, [
+        lambda: rf2.predict_mask(q, k, gnp, sparsity, wl.sink, kmax=kept, ws=ws, out=(idx, cnt), raster=True),
+        lambda: rf2.sparse_attn(q, k, v, idx, cnt, gnp, out=o, raster=True)])
+    flop = 4.0 * gnp.blk * gnp.blk * gnp.D * float(cnt.sum().item())
+    out["no_permute"] = {"blocks": gnp.Nb, "kept": kept, "predict_mask_ms": t_mask, "sparse_attn_ms": t_attn,
+                         "kept_TFLOP/s": flop / (t_attn * 1e-3) / 1e12}
+    del idx, cnt, ws
+    for name, prm in (("rf1", rf2.V1Params()), ("rf1_plus", rf2.V1Params(dynamic=True)),
+                      ("rf1_alpha0.3", rf2.V1Params(alpha=0.3))):
+        ws = torch.empty(rf2.v1_workspace_size(g, prm), dtype=torch.uint8, device=dev)
+        res = {}
+
+        def predict():
+            res["lists"] = rf2.v1_predict_mask(q, k, g, prm, ws=ws)
+
+        def attend():
+            idx1, cnt1 = res["lists"][:2]
+            rf2.sparse_attn(q, k, v, idx1, cnt1, g, out=o, raster=True)
+
+        t_pred, t_attn = _time_legs(stream, iters, [predict, attend])
+        idx1, cnt1, cls, _ = res["lists"]
+        flop = 4.0 * g.blk * g.blk * g.D * float(cnt1.sum().item())
+        out[name] = {"params": dataclasses_asdict(prm), "v1_predict_mask_ms": t_pred, "sparse_attn_ms": t_attn,
+                     "classes_t_s_x": np.bincount(cls.cpu().numpy().reshape(-1), minlength=3).tolist(),
+                     "mean_kept": float(cnt1.float().mean().item()), "blocks": g.Nb,
+                     "kept_TFLOP/s": flop / (t_attn * 1e-3) / 1e12}
+    return out
+
+
+def dataclasses_asdict(x):
+    import dataclasses
+
+    return dataclasses.asdict(x)
 
 
 def main():
@@ -376,6 +444,9 @@ def main():
                "pipelined": "copies of neighbouring calls overlap the call's compute (2 copy streams)"}
         del ws, din, dout
 
+    variants = None if a.no_variants else run_variants(rf2, g, wl, sparsity, q, k, v, o, stream, dev,
+                                                        iters=max(3, min(a.steps, 5)))
+
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         cb = run_cpu_baseline(wl, sparsity, a.cpu_seconds)
@@ -416,6 +487,7 @@ def main():
         "gpu_launches": launches_per_step * a.steps,
         "e2e": e2e,
         "cpu_baseline": cpu,
+        "variants": variants,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -18,11 +18,14 @@
 //   arm_recall_kernel : one CTA per (128 sampled queries, sample, b*heads).  TMA brings
 //                       the query tile once and key tiles through a 2-stage ring; one
 //                       thread issues the 128x128 products into a double-buffered TMEM
-//                       accumulator; four warps read their rows back and keep, per row,
-//                       an online softmax with the total mass and the mass inside four
-//                       band radii (the static bandwidth and the three RainFusion+ ones).
-//                       Each warp writes the sum over its rows of inside / total.  Key
-//                       coordinates come from a table built by arm_coords_kernel.
+//                       accumulator; eight warps read the rows back (two per TMEM lane
+//                       quarter, one per column half) and keep, per row, an online
+//                       softmax with the total mass and the mass inside four band radii
+//                       (the static bandwidth and the three RainFusion+ ones); a chunk of
+//                       32 keys in one window takes one band test.  The halves are merged
+//                       and each warp of the first half writes the sum over its rows of
+//                       inside / total.  Key coordinates come from a table built by
+//                       arm_coords_kernel.
 //   arm_finalize_kernel: per (b, head) the recall (rows summed in a fixed order), the
 //                       class and the band radius or stride.
 //   rf1_lists_kernel   : one warp per (b, head, query block): ascending kept list by
@@ -36,7 +39,8 @@ namespace rf2 {
 namespace {
 
 constexpr int kATile = 128;           // sampled queries per CTA, keys per tile
-constexpr int kAThreads = 160;        // warps 0-3: rows; warp 4: TMA and MMA issue
+constexpr int kAWarpsRows = 8;        // warps 0-7: rows (lane quarter w % 4, column half w / 4)
+constexpr int kAThreads = 32 * kAWarpsRows + 32;  // + warp 8: TMA and MMA issue
 constexpr int kATmemCols = 2 * kATile;
 constexpr uint64_t kArmWaitNs = 500ull * 1000ull * 1000ull;
 
@@ -56,7 +60,7 @@ struct ArmCfg {
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kChunks * kTileBytes;        // 2 stages x kChunks slices
   static constexpr int kOffBar = kOffK + 2 * kChunks * kTileBytes;
-  static constexpr int kUsed = kOffBar + 64 + 1024;         // + alignment slack
+  static constexpr int kUsed = kOffBar + 64 + kATile * 7 * 4 + 1024;  // + merge rows, alignment slack
   // at most two CTAs per SM, so that their TMEM (256 columns each) always fits
   static constexpr int kSmem = kUsed > 80 * 1024 ? kUsed : 80 * 1024;
 };
@@ -114,7 +118,7 @@ __global__ void __launch_bounds__(kAThreads) arm_recall_kernel(const __grid_cons
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(bar_kfull + 8 * s, 1);
       ptx::mbar_init(bar_acc + 8 * s, 1);
-      ptx::mbar_init(bar_free + 8 * s, 4);
+      ptx::mbar_init(bar_free + 8 * s, kAWarpsRows);
     }
     ptx::mbar_init(bar_done, 1);
     abort_s = 0;
@@ -126,7 +130,7 @@ __global__ void __launch_bounds__(kAThreads) arm_recall_kernel(const __grid_cons
   const uint32_t tmem = tmem_slot;
   volatile int* abort_flag = &abort_s;
 
-  if (warp == 4) {
+  if (warp == kAWarpsRows) {
     if (lane == 0) {
       ptx::prefetch_tmap(mq);
       ptx::prefetch_tmap(mk);
@@ -185,9 +189,11 @@ __global__ void __launch_bounds__(kAThreads) arm_recall_kernel(const __grid_cons
       ptx::mbar_wait(bar_done, 0, nullptr, nullptr, kArmWaitNs, 0);
     }
   } else {
-    // rows: thread r owns sampled query qt * 128 + r (TMEM lane r).  No CTA-wide barrier
-    // inside the loop: a warp that gives up leaves without waiting for the others.
-    const int r = threadIdx.x;
+    // rows: warp w reads TMEM lanes 32 (w % 4) .. + 31 (query qt * 128 + r) and keeps an
+    // online softmax over the key columns of its half (w / 4) of every tile.  No CTA-wide
+    // barrier inside the loop: a warp that gives up leaves without waiting for the others.
+    const int lq = warp & 3, half = warp >> 2;
+    const int r = lq * 32 + lane;
     const int qrow = qt * kATile + r;
     const bool row_valid = qrow < S;
     const int* cs = coords + a.coord_off[p];
@@ -205,12 +211,14 @@ __global__ void __launch_bounds__(kAThreads) arm_recall_kernel(const __grid_cons
       ptx::tc_fence_after();
       const int nvalid = min(kATile, S - kt * kATile);
 #pragma unroll 1
-      for (int c = 0; c * 32 < nvalid; ++c) {
+      for (int c = half * 2; c < half * 2 + 2 && c * 32 < nvalid; ++c) {
         const int nv = min(32, nvalid - c * 32);
-        // lane e holds the coordinate of key c * 32 + e; broadcast by shuffles below
+        // lane e holds the coordinate of key c * 32 + e
         const int ck = lane < nv ? __ldg(cs + kt * kATile + c * 32 + lane) : 0;
+        const int ck0 = __shfl_sync(0xffffffffu, ck, 0);
+        const bool uniform = __all_sync(0xffffffffu, lane >= nv || ck == ck0);
         uint32_t v[32];
-        ptx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(st * kATile + c * 32), v);
+        ptx::tmem_ld32(tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)(st * kATile + c * 32), v);
         float cm = -INFINITY;
 #pragma unroll
         for (int e = 0; e < 32; ++e)
@@ -223,15 +231,27 @@ __global__ void __launch_bounds__(kAThreads) arm_recall_kernel(const __grid_cons
           for (int l = 0; l < 4; ++l) in[l] *= f;
           m = cm;
         }
+        if (uniform) {
+          // every key of the chunk has the same window: one band test for the chunk
+          float csum = 0.f;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int cke = __shfl_sync(0xffffffffu, ck, e);
-          if (e < nv) {
-            const float x = ptx::ex2(fmaf(__uint_as_float(v[e]), a.scale_log2, -m));
-            tot += x;
-            const int d = abs(cq - cke);
+          for (int e = 0; e < 32; ++e)
+            if (e < nv) csum += ptx::ex2(fmaf(__uint_as_float(v[e]), a.scale_log2, -m));
+          tot += csum;
+          const int d = abs(cq - ck0);
 #pragma unroll
-            for (int l = 0; l < 4; ++l) in[l] += d <= R[l] ? x : 0.f;
+          for (int l = 0; l < 4; ++l) in[l] += d <= R[l] ? csum : 0.f;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int cke = __shfl_sync(0xffffffffu, ck, e);
+            if (e < nv) {
+              const float x = ptx::ex2(fmaf(__uint_as_float(v[e]), a.scale_log2, -m));
+              tot += x;
+              const int d = abs(cq - cke);
+#pragma unroll
+              for (int l = 0; l < 4; ++l) in[l] += d <= R[l] ? x : 0.f;
+            }
           }
         }
       }
@@ -239,20 +259,41 @@ __global__ void __launch_bounds__(kAThreads) arm_recall_kernel(const __grid_cons
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar_free + 8 * st);
     }
-    // per warp: sum of inside / total over its valid rows (fixed shuffle order)
-    float ratio[4];
+    // Merge the two column halves of each row (every row thread reaches this barrier
+    // exactly once, whether or not its loop gave up), then per warp of the first half:
+    // the sum of inside / total over its valid rows, in a fixed shuffle order.
+    float* mrg = reinterpret_cast<float*>(smem + C::kOffBar + 64);  // [128 rows][7]
+    if (half == 1) {
+      float* o = mrg + r * 7;
+      o[0] = m; o[1] = tot;
 #pragma unroll
-    for (int l = 0; l < 4; ++l) {
-      ratio[l] = (ok && row_valid && tot > 0.f) ? in[l] / tot : 0.f;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ratio[l] += __shfl_xor_sync(0xffffffffu, ratio[l], o);
+      for (int l = 0; l < 4; ++l) o[2 + l] = in[l];
+      o[6] = ok ? 1.f : 0.f;
     }
-    if (lane < 4) {
-      float v = ratio[0];
-      if (lane == 1) v = ratio[1];
-      if (lane == 2) v = ratio[2];
-      if (lane == 3) v = ratio[3];
-      partial[((((long long)bh * 2 + p) * a.tiles_max + qt) * 4 + warp) * 4 + lane] = v;
+    ptx::named_bar_sync(1, 32 * kAWarpsRows);
+    if (half == 0) {
+      const float* o = mrg + r * 7;
+      const float m1 = o[0];
+      const float mm = fmaxf(m, m1);
+      const float f0 = ptx::ex2(m - mm), f1 = ptx::ex2(m1 - mm);
+      tot = tot * f0 + o[1] * f1;
+#pragma unroll
+      for (int l = 0; l < 4; ++l) in[l] = in[l] * f0 + o[2 + l] * f1;
+      ok = ok && o[6] != 0.f;
+      float ratio[4];
+#pragma unroll
+      for (int l = 0; l < 4; ++l) {
+        ratio[l] = (ok && row_valid && tot > 0.f) ? in[l] / tot : 0.f;
+#pragma unroll
+        for (int sh = 16; sh > 0; sh >>= 1) ratio[l] += __shfl_xor_sync(0xffffffffu, ratio[l], sh);
+      }
+      if (lane < 4) {
+        float v = ratio[0];
+        if (lane == 1) v = ratio[1];
+        if (lane == 2) v = ratio[2];
+        if (lane == 3) v = ratio[3];
+        partial[((((long long)bh * 2 + p) * a.tiles_max + qt) * 4 + lq) * 4 + lane] = v;
+      }
     }
   }
   ptx::tc_fence_before();
