@@ -22,7 +22,7 @@ from ._lib import RF2_CHECKED, RF2_SINK_ADDITIVE, Rf2Geom
 __all__ = [
     "Geometry", "Rf2Error", "permute", "unpermute", "kept_count", "workspace_size",
     "predict_mask", "sparse_attn", "attention", "library", "Schedule", "StepAttention",
-    "V1Params", "v1_kmax", "v1_workspace_size", "v1_predict_mask",
+    "V1Params", "v1_kmax", "v1_workspace_size", "v1_predict_mask", "quantize_fp8", "sparse_attn_fp8",
 ]
 
 
@@ -202,12 +202,18 @@ def sparse_attn(qp: torch.Tensor, kp: torch.Tensor, vp: torch.Tensor, idx: torch
 def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Geometry, sparsity: float,
               sink: bool = True, scale: float = 0.0, additive: bool = False,
               return_idx: bool = False, checked: bool = False,
-              ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None):
+              ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None, fp8: bool = False):
     """The whole RF2 path on model-order tensors: mask prediction, then block-sparse
-    attention; the window permutation is done by the kernels' gathers and scatters."""
+    attention; the window permutation is done by the kernels' gathers and scatters.
+    fp8: quantise Q, K, V to e4m3 after the mask prediction and attend on e4m3 operands."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _cuda_bf16(t, n, (g.B, g.N, g.heads, g.D))
-    nbytes = workspace_size(g, sparsity, sink, additive, attention=True)
+    extra = _lib.RF2_FP8 if fp8 else 0
+    cg0 = g.c()
+    nbytes = library().rf2_workspace_size(ctypes.byref(cg0), float(sparsity), int(sink),
+                                          _flags(g, additive, False) | extra, 1)
+    if nbytes == 0:
+        raise Rf2Error(_lib.RF2_ERR_INVALID_ARG, "rf2_workspace_size")
     if ws is None or ws.numel() < nbytes:
         ws = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
     if out is None:
@@ -220,8 +226,48 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Geometry, sp
     _check(library().rf2_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(cg),
                                    float(sparsity), int(sink), float(scale), out.data_ptr(),
                                    0 if idx is None else idx.data_ptr(), ws.data_ptr(), ws.numel(),
-                                   _flags(g, additive, checked), _stream(q)), "rf2_attention")
+                                   _flags(g, additive, checked) | extra, _stream(q)), "rf2_attention")
     return (out, idx) if return_idx else out
+
+
+def quantize_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Geometry, out=None):
+    """Per-(batch, head, block) e4m3 quantisation of model-order q, k, v (rf2_quantize_fp8).
+    Returns (q8, k8, v8) uint8 [B, N, heads, D] holding e4m3 codes, and scales
+    [3, B, heads, Nb] float32."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _cuda_bf16(t, n, (g.B, g.N, g.heads, g.D))
+    if out is None:
+        out = tuple(torch.empty((g.B, g.N, g.heads, g.D), dtype=torch.uint8, device=q.device) for _ in range(3)) + (
+            torch.empty((3, g.B, g.heads, g.Nb), dtype=torch.float32, device=q.device),)
+    q8, k8, v8, sc = out
+    cg = g.c()
+    _check(library().rf2_quantize_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(cg), g.flags,
+                                      q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), sc.data_ptr(), _stream(q)),
+           "rf2_quantize_fp8")
+    return q8, k8, v8, sc
+
+
+def sparse_attn_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, scales: torch.Tensor, idx: torch.Tensor,
+                    cnt: torch.Tensor, g: Geometry, scale: float = 0.0, checked: bool = False,
+                    out: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Block-sparse attention over e4m3 operands (rf2_sparse_attn_fp8); model order."""
+    for t, n in ((q8, "q8"), (k8, "k8"), (v8, "v8")):
+        if not t.is_cuda or t.dtype != torch.uint8 or tuple(t.shape) != (g.B, g.N, g.heads, g.D) or not t.is_contiguous():
+            raise ValueError(f"{n}: expected contiguous CUDA uint8 {(g.B, g.N, g.heads, g.D)}")
+    if scales.dtype != torch.float32 or tuple(scales.shape) != (3, g.B, g.heads, g.Nb):
+        raise ValueError("scales: expected float32 [3, B, heads, Nb]")
+    if idx.dtype != torch.int32 or cnt.dtype != torch.int32 or not idx.is_contiguous():
+        raise ValueError("idx and cnt must be contiguous int32")
+    if out is None:
+        out = torch.empty((g.B, g.N, g.heads, g.D), dtype=torch.bfloat16, device=q8.device)
+    if status is None and checked:
+        status = torch.zeros(1, dtype=torch.int32, device=q8.device)
+    cg = g.c()
+    _check(library().rf2_sparse_attn_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), scales.data_ptr(),
+                                         idx.data_ptr(), cnt.data_ptr(), idx.shape[-1], ctypes.byref(cg),
+                                         float(scale), out.data_ptr(), 0 if status is None else status.data_ptr(),
+                                         _flags(g, False, checked), _stream(q8)), "rf2_sparse_attn_fp8")
+    return out
 
 
 @dataclasses.dataclass(frozen=True)

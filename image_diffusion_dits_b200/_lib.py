@@ -20,6 +20,7 @@ RF2_SINK_ADDITIVE = 1
 RF2_CHECKED = 2
 RF2_RASTER = 4
 RF2_NO_PERMUTE = 8
+RF2_FP8 = 16
 RF2_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 # Every symbol include/rf2.h declares.
@@ -33,6 +34,8 @@ EXPORTS = (
     "rf2_sparse_attn",
     "rf2_attention",
     "rf2_schedule_action",
+    "rf2_quantize_fp8",
+    "rf2_sparse_attn_fp8",
     "rf2_v1_kmax",
     "rf2_v1_workspace_size",
     "rf2_v1_predict_mask",
@@ -82,6 +85,9 @@ _SIGS = {
     "rf2_attention": (ctypes.c_int, [_vp, _vp, _vp, _gp, ctypes.c_double, ctypes.c_int, ctypes.c_float,
                                      _vp, _i32p, _vp, ctypes.c_size_t, ctypes.c_uint, _vp]),
     "rf2_schedule_action": (ctypes.c_int, [ctypes.POINTER(Rf2Schedule), ctypes.c_int]),
+    "rf2_quantize_fp8": (ctypes.c_int, [_vp, _vp, _vp, _gp, ctypes.c_uint, _vp, _vp, _vp, _vp, _vp]),
+    "rf2_sparse_attn_fp8": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32p, _i32p, ctypes.c_int, _gp, ctypes.c_float,
+                                           _vp, _i32p, ctypes.c_uint, _vp]),
     "rf2_v1_kmax": (ctypes.c_int, [_gp, ctypes.POINTER(Rf2V1Params), ctypes.c_uint]),
     "rf2_v1_workspace_size": (ctypes.c_size_t, [_gp, ctypes.POINTER(Rf2V1Params), ctypes.c_uint]),
     "rf2_v1_predict_mask": (ctypes.c_int, [_vp, _vp, _gp, ctypes.POINTER(Rf2V1Params), ctypes.c_uint, _i32p,

@@ -69,10 +69,12 @@ MaskWs mask_ws_layout(const Geo& g, uint8_t* base) {
 struct AttnWs {
   MaskWs mask;
   int32_t *idx, *cnt;
+  uint8_t *q8, *k8, *v8;  // RF2_FP8: e4m3 copies of Q, K, V
+  float* scales;          // RF2_FP8: [3][B][heads][Nb]
   size_t bytes;
 };
 
-AttnWs attn_ws_layout(const Geo& g, int kept, uint8_t* base) {
+AttnWs attn_ws_layout(const Geo& g, int kept, uint8_t* base, unsigned flags = 0) {
   AttnWs w;
   w.mask = mask_ws_layout(g, base);
   size_t off = w.mask.bytes;
@@ -80,6 +82,17 @@ AttnWs attn_ws_layout(const Geo& g, int kept, uint8_t* base) {
   off += align_up((size_t)g.B * g.heads * g.Nb * kept * sizeof(int32_t));
   w.cnt = reinterpret_cast<int32_t*>(base + off);
   off += align_up((size_t)g.B * g.heads * g.Nb * sizeof(int32_t));
+  w.q8 = w.k8 = w.v8 = nullptr;
+  w.scales = nullptr;
+  if (flags & RF2_FP8) {
+    const size_t t8 = align_up((size_t)g.B * g.N * g.heads * g.D);
+    w.q8 = base + off;
+    w.k8 = base + off + t8;
+    w.v8 = base + off + 2 * t8;
+    off += 3 * t8;
+    w.scales = reinterpret_cast<float*>(base + off);
+    off += align_up((size_t)3 * g.B * g.heads * g.Nb * sizeof(float));
+  }
   w.bytes = off;
   return w;
 }
@@ -180,6 +193,46 @@ size_t v1_ws_bytes(const V1Call& c) {
 
 extern "C" {
 
+int rf2_quantize_fp8(const void* q, const void* k, const void* v, const rf2_geom* g, unsigned flags,
+                     void* q8, void* k8, void* v8, float* scales, void* stream) {
+  int st = check_geom(g, flags);
+  if (st != RF2_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || q8 == nullptr || k8 == nullptr || v8 == nullptr ||
+      scales == nullptr)
+    return RF2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q8) || !aligned16(k8) || !aligned16(v8) ||
+      ((uintptr_t)scales & 3u))
+    return RF2_ERR_ALIGNMENT;
+  Geo geo = rf2::make_call_geo(*g, flags);
+  log_geo("quantize_fp8", geo, 0);
+  cudaError_t e = rf2::launch_quant_fp8(q, k, v, static_cast<uint8_t*>(q8), static_cast<uint8_t*>(k8),
+                                        static_cast<uint8_t*>(v8), scales, geo, (cudaStream_t)stream);
+  if (e == cudaErrorNotSupported) return RF2_ERR_UNSUPPORTED;
+  return cuda_status(e);
+}
+
+int rf2_sparse_attn_fp8(const void* q8, const void* k8, const void* v8, const float* scales,
+                        const int32_t* idx, const int32_t* cnt, int kmax, const rf2_geom* g, float scale,
+                        void* o, int32_t* status, unsigned flags, void* stream) {
+  int st = check_geom(g, flags);
+  if (st != RF2_OK) return st;
+  if (q8 == nullptr || k8 == nullptr || v8 == nullptr || scales == nullptr || idx == nullptr || cnt == nullptr ||
+      o == nullptr || kmax < 1 || !isfinite(scale) || scale < 0.f)
+    return RF2_ERR_INVALID_ARG;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o) || ((uintptr_t)scales & 3u) ||
+      ((uintptr_t)idx & 3u) || ((uintptr_t)cnt & 3u) || ((uintptr_t)status & 3u))
+    return RF2_ERR_ALIGNMENT;
+  Geo geo = rf2::make_call_geo(*g, flags);
+  const float sc = scale == 0.f ? (float)(1.0 / sqrt((double)geo.D)) : scale;
+  log_geo("sparse_attn_fp8", geo, kmax);
+  cudaError_t e = rf2::launch_sparse_attn_fp8(static_cast<const uint8_t*>(q8), static_cast<const uint8_t*>(k8),
+                                              static_cast<const uint8_t*>(v8), scales, idx, cnt, kmax, geo, sc, o,
+                                              status, (cudaStream_t)stream);
+  if (e == cudaErrorNotSupported) return RF2_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return RF2_ERR_CUDA;
+  return finish_checked(flags, status, (cudaStream_t)stream);
+}
+
 int rf2_v1_kmax(const rf2_geom* g, const rf2_v1_params* p, unsigned flags) {
   V1Call c;
   int st = v1_prepare(g, p, flags, &c);
@@ -277,7 +330,7 @@ size_t rf2_workspace_size(const rf2_geom* g, double sparsity, int sink, unsigned
   if (!(sparsity >= 0.0 && sparsity <= 1.0)) return 0;
   Geo geo = rf2::make_call_geo(*g, flags);
   if (!attention) return mask_ws_layout(geo, nullptr).bytes;
-  return attn_ws_layout(geo, kept_of(geo, sparsity, sink, flags), nullptr).bytes;
+  return attn_ws_layout(geo, kept_of(geo, sparsity, sink, flags), nullptr, flags).bytes;
 }
 
 static int predict_mask_impl(const void* qp, const void* kp, const Geo& geo, double sparsity,
@@ -350,7 +403,8 @@ int rf2_attention(const void* q, const void* k, const void* v, const rf2_geom* g
   if (!aligned16(ws)) return RF2_ERR_ALIGNMENT;
   Geo geo = rf2::make_call_geo(*g, flags);
   const int kept = kept_of(geo, sparsity, sink, flags);
-  AttnWs w = attn_ws_layout(geo, kept, static_cast<uint8_t*>(ws));
+  if ((flags & RF2_FP8) && (geo.D != 128 || geo.blk != 128)) return RF2_ERR_UNSUPPORTED;
+  AttnWs w = attn_ws_layout(geo, kept, static_cast<uint8_t*>(ws), flags);
   if (ws_bytes < w.bytes) return RF2_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
   const float sc = scale == 0.f ? (float)(1.0 / sqrt((double)geo.D)) : scale;
@@ -360,7 +414,13 @@ int rf2_attention(const void* q, const void* k, const void* v, const rf2_geom* g
   if (e != cudaSuccess) return RF2_ERR_CUDA;
   st = predict_mask_impl(q, k, geo, sparsity, sink, flags | RF2_RASTER, w.idx, w.cnt, kept, w.mask, s);
   if (st != RF2_OK) return st;
-  e = rf2::launch_sparse_attn(q, k, v, w.idx, w.cnt, kept, geo, sc, o, w.mask.status, true, s);
+  if (flags & RF2_FP8) {
+    e = rf2::launch_quant_fp8(q, k, v, w.q8, w.k8, w.v8, w.scales, geo, s);
+    if (e == cudaSuccess)
+      e = rf2::launch_sparse_attn_fp8(w.q8, w.k8, w.v8, w.scales, w.idx, w.cnt, kept, geo, sc, o, w.mask.status, s);
+  } else {
+    e = rf2::launch_sparse_attn(q, k, v, w.idx, w.cnt, kept, geo, sc, o, w.mask.status, true, s);
+  }
   if (e == cudaErrorNotSupported) return RF2_ERR_UNSUPPORTED;
   if (e == cudaSuccess && idx_out != nullptr)
     e = cudaMemcpyAsync(idx_out, w.idx, (size_t)geo.B * geo.heads * geo.Nb * kept * sizeof(int32_t),

@@ -186,6 +186,15 @@ cudaError_t launch_sparse_attn(const void* qp, const void* kp, const void* vp,
                                const int32_t* idx, const int32_t* cnt, int kmax, const Geo& g,
                                float scale, void* op, int32_t* status, bool raster, cudaStream_t s);
 
+// e4m3 variant: per-(batch, head, block) quantisation of model-order Q, K, V into e4m3
+// model-order tensors and scales [3][B][heads][Nb]; attention over them (D = 128,
+// 128-token blocks, model order; cudaErrorNotSupported otherwise).
+cudaError_t launch_quant_fp8(const void* q, const void* k, const void* v, uint8_t* q8, uint8_t* k8, uint8_t* v8,
+                             float* scales, const Geo& g, cudaStream_t s);
+cudaError_t launch_sparse_attn_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, const float* scales,
+                                   const int32_t* idx, const int32_t* cnt, int kmax, const Geo& g, float scale,
+                                   void* op, int32_t* status, cudaStream_t s);
+
 // RainFusion v1: ARM recall of the two samples, head classes, kept lists.  q, k in model
 // order [B, N, heads, D].  cls_out [B*heads] and recall_out [B*heads][2][4] may be null.
 cudaError_t launch_rf1(const void* q, const void* k, const Geo& g, const Rf1Args& a, const Rf1Scratch& w,

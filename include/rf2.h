@@ -75,7 +75,10 @@ enum rf2_flags {
      * first-frame sink becomes the blocks that hold a token of frame 0, the first
      * ceil(H*W/blk) blocks.  rf2_permute and rf2_unpermute take no flags and keep
      * the 3D windows. */
-    RF2_NO_PERMUTE = 8u
+    RF2_NO_PERMUTE = 8u,
+    /* rf2_attention: quantise Q, K and V to e4m3 (rf2_quantize_fp8) after the mask
+     * prediction and attend with rf2_sparse_attn_fp8.  D = 128 and 128-token blocks only. */
+    RF2_FP8 = 16u
 };
 
 /* rf2_permute - 3D window permutation (mlsanity index page, Abstract, insight (2)
@@ -183,11 +186,40 @@ int rf2_sparse_attn(const void* qp, const void* kp, const void* vp, const int32_
  * and row scatters, with no permuted copies).
  *   q, k, v : [B, N, heads, D] bf16 (read).   o : [B, N, heads, D] bf16 (written).
  *   idx_out : optional [B, heads, Nb, kept] int32 copy of the kept lists (may be NULL).
- *   ws, ws_bytes : device scratch of at least rf2_workspace_size(..., 1) bytes.
+ *   ws, ws_bytes : device scratch of at least rf2_workspace_size(..., 1) bytes (with
+ *   RF2_FP8 it also holds the e4m3 copies of Q, K, V and their scales).
  * Errors: as rf2_predict_mask and rf2_sparse_attn. */
 int rf2_attention(const void* q, const void* k, const void* v, const rf2_geom* g,
                   double sparsity, int sink, float scale, void* o, int32_t* idx_out,
                   void* ws, size_t ws_bytes, unsigned flags, void* stream);
+
+/* e4m3 variant of the attention.  The pages suggest combining the block-sparse attention
+ * with quantisation; the FP8 form below is this library's reading.  Every (batch, head,
+ * block) of Q, K and V gets one scale: amax = max |x| over the block's real tokens and
+ * the head's D channels, inv = 448 / amax, scale = amax / 448 (fp32, rounded to
+ * nearest; amax = 0 gives 0 for both); code = e4m3(x * inv) with round to nearest even
+ * and saturation to +-448.
+ *
+ * rf2_quantize_fp8 - q, k, v : [B, N, heads, D] bf16, model order (read).
+ *   q8, k8, v8 : [B, N, heads, D] e4m3 codes, model order (written).
+ *   scales : [3][B][heads][Nb] float (written): Q, K, V scales in that order.
+ *   Every pointer 16-byte aligned.
+ *   flags : RF2_NO_PERMUTE selects raster blocks.  Errors: RF2_ERR_INVALID_ARG,
+ *   RF2_ERR_UNSUPPORTED, RF2_ERR_ALIGNMENT, RF2_ERR_CUDA. */
+int rf2_quantize_fp8(const void* q, const void* k, const void* v, const rf2_geom* g, unsigned flags,
+                     void* q8, void* k8, void* v8, float* scales, void* stream);
+
+/* rf2_sparse_attn_fp8 - block-sparse attention over e4m3 operands (tcgen05 kind::f8f6f4):
+ *   S = (Q8 K8_j^T) * sq * sk_j * scale with fp32 accumulation; P = exp2 of the scores
+ *   minus the running max (fp32 row sums), multiplied by sv_j / max sv over the row's kept
+ *   blocks and rounded to e4m3; O = (sum_j P_j V8_j) * max sv / l, written as bf16.
+ *   q8, k8, v8 : [B, N, heads, 128] e4m3, model order; scales as rf2_quantize_fp8 writes
+ *   them; idx, cnt, kmax, status as rf2_sparse_attn; o : [B, N, heads, 128] bf16.
+ *   D = 128 and 128-token blocks only (else RF2_ERR_UNSUPPORTED).
+ * Errors: as rf2_sparse_attn. */
+int rf2_sparse_attn_fp8(const void* q8, const void* k8, const void* v8, const float* scales,
+                        const int32_t* idx, const int32_t* cnt, int kmax, const rf2_geom* g, float scale,
+                        void* o, int32_t* status, unsigned flags, void* stream);
 
 /* Step schedule of the attention calls of one generation.  RainFusion v1 keeps the first
  * 10 % of the diffusion timesteps dense (pith.science review, "Free parameters": dense
