@@ -473,17 +473,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int q = 0; q < kBLK / 32; ++q) vm[q] = 0xffffffffu;
         }
-        // pass 1: the row max of the raw scores (the scale is positive, so it commutes
-        // with max), from one load of the whole row; the registers are free again after it
+        // the whole S row in one TMEM load; the row max of the raw scores (the scale is
+        // positive, so it commutes with max)
         float mx;
-        {
-          uint32_t tt[kBLK];
-          ptx::tmem_ld32x128(srow, tt);
-          if (partial) {
+        uint32_t tt[kBLK];
+        ptx::tmem_ld32x128(srow, tt);
+        if (partial) {
 #pragma unroll
-            for (int c = 0; c < kBLK; ++c)
-              if (!((vm[c >> 5] >> (c & 31)) & 1u)) tt[c] = __float_as_uint(-INFINITY);
-          }
+          for (int c = 0; c < kBLK; ++c)
+            if (!((vm[c >> 5] >> (c & 31)) & 1u)) tt[c] = __float_as_uint(-INFINITY);
+        }
+        {
           float mx8[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(tt[e]);
@@ -515,27 +515,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tmem_st32(orow_t + c * 32, tt);
           }
         }
-        // p = exp2(x * sc - m) in packed f16 (arguments from one packed fp32 FMA per pair);
-        // P = e4m3(p * sv_j / vmax) from f16x2; the row sum adds the f16 values of each
-        // 16-column chunk in f16x2 and widens once per chunk.  P goes to shared memory in
-        // the 128-byte swizzle: 16-byte chunk ch of row r at chunk ch ^ (r % 8).
-        // pass 2, 32 columns at a time: p = exp2(x * sc - m) in packed f16 (arguments from
-        // one packed fp32 FMA per pair), P = e4m3(p * sv_j / vmax) from f16x2, four codes
-        // per word; the row sum adds the f16 values of 16 columns in f16x2 and widens once.
+        // 32 columns at a time: p = exp2(x * sc - m) in packed f16 (arguments from one packed
+        // fp32 FMA per pair), P = e4m3(p * sv_j / vmax) from f16x2, four codes per word; the
+        // row sum adds the f16 values of 16 columns in f16x2 and widens once.
         const uint64_t sc2 = ptx::f2(sc, sc), nm2 = ptx::f2(-m_run, -m_run);
         const uint32_t vs2 = f16x2_from(vsc_s[i], vsc_s[i]);
         float lsum = 0.f;
-#pragma unroll 1
+#pragma unroll
         for (int q = 0; q < kBLK / 32; ++q) {
           uint32_t pk[8];
-          uint32_t tt[32];
-          ptx::tmem_ld32(srow + q * 32, tt);
-          if (partial) {
-            const uint32_t mq = vm[q];
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (!((mq >> e) & 1u)) tt[e] = __float_as_uint(-INFINITY);
-          }
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             uint32_t e2[8];
@@ -543,8 +531,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int qd = 0; qd < 8; ++qd) {
               const int c = half * 16 + qd * 2;
               float a0, a1;
-              ptx::f2split(ptx::ffma2(ptx::f2(__uint_as_float(tt[c]), __uint_as_float(tt[c + 1])), sc2, nm2), a0,
-                           a1);
+              const uint64_t xx = ptx::f2(__uint_as_float(tt[q * 32 + c]), __uint_as_float(tt[q * 32 + c + 1]));
+              ptx::f2split(ptx::ffma2(xx, sc2, nm2), a0, a1);
               e2[qd] = ex2_h2(f16x2_from(a0, a1));
             }
 #pragma unroll
@@ -554,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             lsum += h2_sum_f32(hadd2(hadd2(hadd2(e2[0], e2[1]), hadd2(e2[2], e2[3])),
                                      hadd2(hadd2(e2[4], e2[5]), hadd2(e2[6], e2[7]))));
           }
-          // P columns 8q .. 8q+7 lie in S columns this thread has already read
+          // P columns 8q .. 8q+7 over S columns already loaded into registers
           tmem_st8(srow + q * 8, pk);
         }
         ptx::tmem_wait_st();
