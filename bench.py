@@ -236,6 +236,29 @@ def run_variants(rf2, g, wl, sparsity, q, k, v, o, stream, dev, iters):
     out["no_permute"] = {"blocks": gnp.Nb, "kept": kept, "predict_mask_ms": t_mask, "sparse_attn_ms": t_attn,
                          "kept_TFLOP/s": flop / (t_attn * 1e-3) / 1e12}
     del idx, cnt, ws
+    # e4m3 operands: quantisation, then the attention over the same kept lists as the
+    # headline step (lists from the bf16 mask prediction)
+    if g.D == 128 and g.blk == 128:
+        kept = rf2.kept_count(g, sparsity, wl.sink)
+        idx = torch.empty((g.B, g.heads, g.Nb, kept), dtype=torch.int32, device=dev)
+        cnt = torch.empty((g.B, g.heads, g.Nb), dtype=torch.int32, device=dev)
+        rf2.predict_mask(q, k, g, sparsity, wl.sink, kmax=kept, out=(idx, cnt), raster=True)
+        q8s = rf2.quantize_fp8(q, k, v, g)
+        t_quant, t_attn = _time_legs(stream, iters, [
+            lambda: rf2.quantize_fp8(q, k, v, g, out=q8s),
+            lambda: rf2.sparse_attn_fp8(*q8s, idx, cnt, g, out=o)])
+        flop = 4.0 * g.blk * g.blk * g.D * float(cnt.sum().item())
+        peaks = _peaks()
+        achieved = flop / (t_attn * 1e-3) / 1e12
+        # algorithmic HBM bytes of the quantisation: bf16 Q, K, V read once, e4m3 written
+        qbytes = 3 * (g.B * g.N * g.heads * g.D) * (2 + 1)
+        out["fp8"] = {"quantize_ms": t_quant, "quantize_bytes": qbytes,
+                      "quantize_GB/s": qbytes / (t_quant * 1e-3) / 1e9,
+                      "sparse_attn_fp8_ms": t_attn, "kept_TFLOP/s": achieved,
+                      "roofline": {"bound": "tensor", "achieved": achieved, "peak": 2 * peaks["bf16_tflops"],
+                                   "unit": "TFLOP/s", "frac": achieved / (2 * peaks["bf16_tflops"]),
+                                   "peak_source": peaks["source"] + " burst bf16 x 2 (nominal fp8/bf16 ratio)"}}
+        del q8s, idx, cnt
     for name, prm in (("rf1", rf2.V1Params()), ("rf1_plus", rf2.V1Params(dynamic=True)),
                       ("rf1_alpha0.3", rf2.V1Params(alpha=0.3))):
         ws = torch.empty(rf2.v1_workspace_size(g, prm), dtype=torch.uint8, device=dev)
