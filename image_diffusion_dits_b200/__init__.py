@@ -289,47 +289,6 @@ class Schedule:
         return a
 
 
-class StepAttention:
-    """Block-sparse attention of one generation under a Schedule, on model-order tensors:
-    dense steps attend to every block, predict steps run the mask prediction of their layer
-    and attend with it, reuse steps attend with the layer's last predicted lists.  Every
-    step runs on the library's kernels (rf2_predict_mask, rf2_sparse_attn with RF2_RASTER)."""
-
-    def __init__(self, g: Geometry, sparsity: float, sink: bool = True, schedule: Optional[Schedule] = None,
-                 additive: bool = False):
-        self.g, self.sparsity, self.sink, self.additive = g, float(sparsity), bool(sink), bool(additive)
-        self.schedule = schedule if schedule is not None else Schedule(1, 0.0, 1)
-        self.kept = kept_count(g, sparsity, sink, additive)
-        self._lists = {}   # layer -> (idx, cnt) of its last prediction
-        self._dense = None
-        self._ws = None
-
-    def lists(self, layer):
-        """The kept lists (idx, cnt) the layer's last predict step produced."""
-        return self._lists[layer]
-
-    def __call__(self, layer, step: int, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
-                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
-        g = self.g
-        act = self.schedule.action(step)
-        if act == _lib.RF2_STEP_DENSE:
-            if self._dense is None:
-                idx = torch.arange(g.Nb, dtype=torch.int32, device=q.device).expand(g.B, g.heads, g.Nb, g.Nb)
-                cnt = torch.full((g.B, g.heads, g.Nb), g.Nb, dtype=torch.int32, device=q.device)
-                self._dense = (idx.contiguous(), cnt)
-            return sparse_attn(q, k, v, *self._dense, g, out=out, raster=True)
-        if act == _lib.RF2_STEP_PREDICT:
-            if self._ws is None:
-                self._ws = torch.empty(workspace_size(g, self.sparsity, self.sink, self.additive, attention=False),
-                                       dtype=torch.uint8, device=q.device)
-            buf = self._lists.get(layer)
-            self._lists[layer] = predict_mask(q, k, g, self.sparsity, self.sink, self.additive, kmax=self.kept,
-                                              ws=self._ws, out=buf, raster=True)
-        elif layer not in self._lists:
-            raise RuntimeError(f"step {step} reuses the mask of layer {layer!r}, which has none predicted yet")
-        return sparse_attn(q, k, v, *self._lists[layer], g, out=out, raster=True)
-
-
 @dataclasses.dataclass(frozen=True)
 class V1Params:
     """Parameters of the RainFusion v1 mask generators (rf2_v1_params): band half-width as
@@ -389,6 +348,74 @@ def v1_predict_mask(q: torch.Tensor, k: torch.Tensor, g: Geometry, params: V1Par
                                          cls.data_ptr(), rec.data_ptr(), ws.data_ptr(), ws.numel(), _stream(q)),
            "rf2_v1_predict_mask")
     return idx, cnt, cls, rec
+
+
+class StepAttention:
+    """Block-sparse attention of one generation under a Schedule, on model-order tensors:
+    dense steps attend to every block, predict steps run the mask prediction of their layer
+    and attend with it, reuse steps attend with the layer's last predicted lists.
+
+    method: "rf2" predicts with the pooled-score top-k (rf2_predict_mask); "rf1" with the
+    RainFusion v1 generators (rf2_v1_predict_mask, parameters v1_params; sparsity and sink
+    are then unused).  fp8: every step quantises its Q, K, V to e4m3 (rf2_quantize_fp8) and
+    attends with rf2_sparse_attn_fp8.  Every step runs on the library's kernels."""
+
+    def __init__(self, g: Geometry, sparsity: float = 0.8, sink: bool = True, schedule: Optional[Schedule] = None,
+                 additive: bool = False, method: str = "rf2", v1_params: Optional[V1Params] = None,
+                 fp8: bool = False):
+        if method not in ("rf2", "rf1"):
+            raise ValueError("method must be 'rf2' or 'rf1'")
+        self.g, self.sparsity, self.sink, self.additive = g, float(sparsity), bool(sink), bool(additive)
+        self.method, self.fp8 = method, bool(fp8)
+        self.v1_params = v1_params if v1_params is not None else V1Params()
+        self.schedule = schedule if schedule is not None else Schedule(1, 0.0, 1)
+        self.kept = (kept_count(g, sparsity, sink, additive) if method == "rf2" else v1_kmax(g, self.v1_params))
+        self._lists = {}   # layer -> (idx, cnt) of its last prediction
+        self._classes = {}  # layer -> head classes of its last v1 prediction
+        self._dense = None
+        self._ws = None
+        self._q8 = None
+
+    def lists(self, layer):
+        """The kept lists (idx, cnt) the layer's last predict step produced."""
+        return self._lists[layer]
+
+    def head_classes(self, layer):
+        """The RainFusion v1 head classes [B, heads] of the layer's last predict step."""
+        return self._classes[layer]
+
+    def _attend(self, q, k, v, idx, cnt, out):
+        if not self.fp8:
+            return sparse_attn(q, k, v, idx, cnt, self.g, out=out, raster=True)
+        self._q8 = quantize_fp8(q, k, v, self.g, out=self._q8)
+        return sparse_attn_fp8(*self._q8, idx, cnt, self.g, out=out)
+
+    def __call__(self, layer, step: int, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        g = self.g
+        act = self.schedule.action(step)
+        if act == _lib.RF2_STEP_DENSE:
+            if self._dense is None:
+                idx = torch.arange(g.Nb, dtype=torch.int32, device=q.device).expand(g.B, g.heads, g.Nb, g.Nb)
+                cnt = torch.full((g.B, g.heads, g.Nb), g.Nb, dtype=torch.int32, device=q.device)
+                self._dense = (idx.contiguous(), cnt)
+            return self._attend(q, k, v, *self._dense, out)
+        if act == _lib.RF2_STEP_PREDICT:
+            if self.method == "rf1":
+                if self._ws is None:
+                    self._ws = torch.empty(v1_workspace_size(g, self.v1_params), dtype=torch.uint8, device=q.device)
+                idx, cnt, cls, _ = v1_predict_mask(q, k, g, self.v1_params, kmax=self.kept, ws=self._ws)
+                self._lists[layer], self._classes[layer] = (idx, cnt), cls
+            else:
+                if self._ws is None:
+                    self._ws = torch.empty(workspace_size(g, self.sparsity, self.sink, self.additive, attention=False),
+                                           dtype=torch.uint8, device=q.device)
+                buf = self._lists.get(layer)
+                self._lists[layer] = predict_mask(q, k, g, self.sparsity, self.sink, self.additive, kmax=self.kept,
+                                                  ws=self._ws, out=buf, raster=True)
+        elif layer not in self._lists:
+            raise RuntimeError(f"step {step} reuses the mask of layer {layer!r}, which has none predicted yet")
+        return self._attend(q, k, v, *self._lists[layer], out)
 
 
 def default_scale(D: int) -> float:

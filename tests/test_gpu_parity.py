@@ -452,3 +452,43 @@ def test_no_permute_wan720p_end_to_end_sampled():
         ref_rows.append(rows[:hi - lo])
         got_rows.append(got[0, lo:hi, h])
     print("wan720p no_permute", stats, assert_close(np.concatenate(got_rows), np.concatenate(ref_rows), "wan720p"))
+
+
+@pytest.mark.parametrize("method,fp8", [("rf1", False), ("rf2", True), ("rf1", True)])
+def test_step_attention_other_generators_and_fp8(method, fp8):
+    """The schedule with the RainFusion v1 generator and/or e4m3 operands: every step equals
+    the direct call sequence it stands for, bit for bit."""
+    wl = WORKLOADS["video480p"]
+    g = rf2.Geometry(**wl.geom())
+    sched = rf2.Schedule(total_steps=4, dense_fraction=0.25, predict_interval=2)      # D P R P
+    p1 = rf2.V1Params(alpha=0.3)
+    sa = rf2.StepAttention(g, 0.5, wl.sink, schedule=sched, method=method, v1_params=p1, fp8=fp8)
+    same = lambda a, b: torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+    def attend(q, k, v, idx, cnt):
+        if not fp8:
+            return rf2.sparse_attn(q, k, v, idx, cnt, g, raster=True)
+        return rf2.sparse_attn_fp8(*rf2.quantize_fp8(q, k, v, g), idx, cnt, g)
+
+    def predict(q, k):
+        if method == "rf1":
+            idx, cnt, _, _ = rf2.v1_predict_mask(q, k, g, p1, kmax=sa.kept)
+            return idx, cnt
+        return rf2.predict_mask(q, k, g, 0.5, wl.sink, raster=True)
+
+    dense = (torch.arange(g.Nb, dtype=torch.int32, device="cuda").expand(g.B, g.heads, g.Nb, g.Nb).contiguous(),
+             torch.full((g.B, g.heads, g.Nb), g.Nb, dtype=torch.int32, device="cuda"))
+    last = None
+    for step in range(4):
+        q, k, v = (to_dev(gen_tensor(g.B, g.T, g.H, g.W, g.heads, g.D, 8000 + 10 * step + i)) for i in range(3))
+        got = sa(0, step, q, k, v)
+        act = sched.action(step)
+        if act == 0:
+            ref = attend(q, k, v, *dense)
+        else:
+            if act == 1:
+                last = predict(q, k)
+            ref = attend(q, k, v, *last)
+        assert same(got, ref), (method, fp8, step)
+    if method == "rf1":
+        assert sa.head_classes(0).shape == (g.B, g.heads)
