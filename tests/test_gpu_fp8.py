@@ -124,3 +124,26 @@ def test_fp8_attention_end_to_end_wan720p_sampled():
     stats = _close(np.concatenate(g_rows), np.concatenate(r_rows), "wan720p fp8")
     gr, er = np.concatenate(g_rows), np.concatenate(e_rows)
     print("wan720p fp8", stats, "vs exact attention: rel-L2 %.3e" % (np.linalg.norm(gr - er) / np.linalg.norm(er)))
+
+
+@pytest.mark.parametrize("shape,no_permute", [
+    (dict(B=2, heads=2, T=3, H=9, W=17, D=128, wt=2, wh=8, ww=8), False),    # one launch per batch
+    (dict(B=1, heads=2, T=3, H=10, W=13, D=128, wt=1, wh=8, ww=16), True),   # raster blocks, tail of 6
+])
+def test_fp8_attention_batches_and_raster_blocks(shape, no_permute):
+    g = rf2.Geometry(**shape, no_permute=no_permute)
+    og = O.geom(**shape, no_permute=no_permute)
+    q, k, v = _bits(g, 1600)
+    qf, kf, vf = (bf16_bits_to_f64(a) for a in (q, k, v))
+    sel = O.predict_mask(O.permute(qf, og), O.permute(kf, og), og, 0.5, True)
+    idx = torch.from_numpy(sel.idx).cuda()
+    cnt = torch.full(sel.idx.shape[:3], sel.kept, dtype=torch.int32, device="cuda")
+    q8, k8, v8, sc = rf2.quantize_fp8(to_dev(q), to_dev(k), to_dev(v), g)
+    got = to_f64(rf2.sparse_attn_fp8(q8, k8, v8, sc, idx, cnt, g, checked=True))
+    quant = F8.quantised_inputs(qf, kf, vf, og)
+    rows = [(b, h, i) for b in range(og.B) for h in range(og.heads) for i in range(og.Nb)]
+    g_rows, r_rows = [], []
+    for b, h, toks, ref in _ref_rows(quant, og, sel, rows):
+        g_rows.append(got[b, toks, h])
+        r_rows.append(ref)
+    print(shape, no_permute, _close(np.concatenate(g_rows), np.concatenate(r_rows), "fp8 attention"))
