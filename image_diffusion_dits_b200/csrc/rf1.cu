@@ -65,14 +65,27 @@ struct ArmCfg {
   static constexpr int kSmem = kUsed > 80 * 1024 ? kUsed : 80 * 1024;
 };
 
-// Window coordinate of every sampled token: sw for the local sample (frame-0 token m),
-// tb for the global sample (raster token m * omega).  coords[a.coord_off[p] + m].
-__global__ void arm_coords_kernel(Rf1Args a, int* __restrict__ coords) {
+// Window coordinate of every sample slot: sw for the local sample, tb for the global one
+// (raster token m * omega); kPadSlot for a pad slot.  coords[a.coord_off[p] + m].  With
+// a.wslots, local slot m is token (dh, dw) = divmod(m % wslots, ww) of frame-0 window
+// sw = m / wslots; otherwise it is frame-0 token m.
+constexpr int kPadSlot = -(1 << 30);
+
+__global__ void arm_coords_kernel(Rf1Args a, int nbh, int* __restrict__ coords) {
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= a.S[0] + a.S[1]) return;
   if (t < a.S[0]) {
-    const int h = t / a.W, w = t - h * a.W;
-    coords[a.coord_off[0] + t] = (h / a.wh) * a.nbw + w / a.ww;
+    int c;
+    if (a.wslots) {
+      const int sw = t / a.wslots, off = t - sw * a.wslots;
+      const int hb = sw / a.nbw, wb = sw - hb * a.nbw;
+      const int h = hb * a.wh + off / a.ww, w = wb * a.ww + off % a.ww;
+      c = (hb < nbh && h < a.HW / a.W && w < a.W) ? sw : kPadSlot;
+    } else {
+      const int h = t / a.W, w = t - h * a.W;
+      c = (h / a.wh) * a.nbw + w / a.ww;
+    }
+    coords[a.coord_off[0] + t] = c;
   } else {
     const long long n = (long long)(t - a.S[0]) * a.omega;
     coords[a.coord_off[1] + t - a.S[0]] = (int)(n / a.HW) / a.wt;
@@ -97,6 +110,20 @@ __global__ void __launch_bounds__(kAThreads) arm_recall_kernel(const __grid_cons
   const int b = bh / a.heads, head = bh - b * a.heads;
   const CUtensorMap* mq = p == 0 ? &tq0 : &tq1;
   const CUtensorMap* mk = p == 0 ? &tk0 : &tk1;
+  // rows r0 .. r0+127 of sample p into a 128-row tile: one 4-D box (sample stride), or,
+  // for the window-ordered local sample, 128 / wslots 5-D window boxes of frame 0
+  const bool windowed = p == 0 && a.wslots > 0;
+  auto load_rows = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, int kc, int r0) {
+    if (windowed) {
+      for (int u = 0; u < kATile / a.wslots; ++u) {
+        const int sw = r0 / a.wslots + u;
+        const int hb = sw / a.nbw, wb = sw - hb * a.nbw;
+        ptx::tma_load_5d(dst + u * a.wslots * 128, map, bar, kc * 64, head, wb * a.ww, hb * a.wh, b * a.T);
+      }
+    } else {
+      tma_load_4d(dst, map, bar, kc * 64, head, r0, b);
+    }
+  };
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -137,14 +164,14 @@ __global__ void __launch_bounds__(kAThreads) arm_recall_kernel(const __grid_cons
       constexpr uint32_t idesc = ptx::idesc_bf16_f32(kATile, kATile, 0);
       ptx::mbar_arrive_expect_tx(bar_q, C::kChunks * C::kTileBytes);
       for (int kc = 0; kc < C::kChunks; ++kc)
-        tma_load_4d(sbase + C::kOffQ + kc * C::kTileBytes, mq, bar_q, kc * 64, head, qt * kATile, b);
+        load_rows(sbase + C::kOffQ + kc * C::kTileBytes, mq, bar_q, kc, qt * kATile);
       int issued[2] = {0, 0}, waited[2] = {0, 0};
       auto load_k = [&](int kt) {
         const int st = kt & 1;
         ptx::mbar_arrive_expect_tx(bar_kfull + 8 * st, C::kChunks * C::kTileBytes);
         for (int kc = 0; kc < C::kChunks; ++kc)
-          tma_load_4d(sbase + C::kOffK + (st * C::kChunks + kc) * C::kTileBytes, mk, bar_kfull + 8 * st,
-                      kc * 64, head, kt * kATile, b);
+          load_rows(sbase + C::kOffK + (st * C::kChunks + kc) * C::kTileBytes, mk, bar_kfull + 8 * st, kc,
+                    kt * kATile);
         ++issued[st];
       };
       for (int kt = 0; kt < 2 && kt < nk; ++kt) load_k(kt);
@@ -195,9 +222,9 @@ __global__ void __launch_bounds__(kAThreads) arm_recall_kernel(const __grid_cons
     const int lq = warp & 3, half = warp >> 2;
     const int r = lq * 32 + lane;
     const int qrow = qt * kATile + r;
-    const bool row_valid = qrow < S;
     const int* cs = coords + a.coord_off[p];
-    const int cq = row_valid ? __ldg(cs + qrow) : 0;
+    const int cq = qrow < S ? __ldg(cs + qrow) : kPadSlot;
+    const bool row_valid = cq != kPadSlot;
     int R[4];
 #pragma unroll
     for (int l = 0; l < 4; ++l) R[l] = a.R[p][l];
@@ -213,16 +240,17 @@ __global__ void __launch_bounds__(kAThreads) arm_recall_kernel(const __grid_cons
 #pragma unroll 1
       for (int c = half * 2; c < half * 2 + 2 && c * 32 < nvalid; ++c) {
         const int nv = min(32, nvalid - c * 32);
-        // lane e holds the coordinate of key c * 32 + e
-        const int ck = lane < nv ? __ldg(cs + kt * kATile + c * 32 + lane) : 0;
+        // lane e holds the coordinate of key c * 32 + e; bit e of live: a real key
+        const int ck = lane < nv ? __ldg(cs + kt * kATile + c * 32 + lane) : kPadSlot;
+        const uint32_t live = __ballot_sync(0xffffffffu, ck != kPadSlot);
         const int ck0 = __shfl_sync(0xffffffffu, ck, 0);
-        const bool uniform = __all_sync(0xffffffffu, lane >= nv || ck == ck0);
+        const bool uniform = live == 0xffffffffu && __all_sync(0xffffffffu, ck == ck0);
         uint32_t v[32];
         ptx::tmem_ld32(tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)(st * kATile + c * 32), v);
         float cm = -INFINITY;
 #pragma unroll
         for (int e = 0; e < 32; ++e)
-          if (e < nv) cm = fmaxf(cm, __uint_as_float(v[e]));
+          if ((live >> e) & 1u) cm = fmaxf(cm, __uint_as_float(v[e]));
         cm *= a.scale_log2;
         if (cm > m) {
           const float f = ptx::ex2(m - cm);
@@ -232,11 +260,10 @@ __global__ void __launch_bounds__(kAThreads) arm_recall_kernel(const __grid_cons
           m = cm;
         }
         if (uniform) {
-          // every key of the chunk has the same window: one band test for the chunk
+          // 32 real keys in one window: one band test for the chunk
           float csum = 0.f;
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (e < nv) csum += ptx::ex2(fmaf(__uint_as_float(v[e]), a.scale_log2, -m));
+          for (int e = 0; e < 32; ++e) csum += ptx::ex2(fmaf(__uint_as_float(v[e]), a.scale_log2, -m));
           tot += csum;
           const int d = abs(cq - ck0);
 #pragma unroll
@@ -245,7 +272,7 @@ __global__ void __launch_bounds__(kAThreads) arm_recall_kernel(const __grid_cons
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int cke = __shfl_sync(0xffffffffu, ck, e);
-            if (e < nv) {
+            if ((live >> e) & 1u) {
               const float x = ptx::ex2(fmaf(__uint_as_float(v[e]), a.scale_log2, -m));
               tot += x;
               const int d = abs(cq - cke);
@@ -317,7 +344,7 @@ __global__ void arm_finalize_kernel(const float* __restrict__ partial, Rf1Args a
       float s = 0.f;
       for (int t = 0; t < tiles; ++t)
         for (int w = 0; w < 4; ++w) s += partial[((((long long)bh * 2 + p) * a.tiles_max + t) * 4 + w) * 4 + l];
-      rec[p][l] = s / (float)a.S[p];
+      rec[p][l] = s / (float)a.S_real[p];
     }
   }
   int cls, prm;
@@ -398,13 +425,31 @@ bool make_sample_map(CUtensorMap* m, const void* base, const Geo& g, int samples
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 5-D view (D, heads, W, H, T*B) of model-order [B, N, heads, D] (the frames of all
+// batches in a row); box = 64 columns x 1 head x one (ww, wh) window of one frame,
+// 128-byte swizzle, zero fill past the grid.
+bool make_frame_window_map(CUtensorMap* m, const void* base, const Geo& g) {
+  EncodeTiledFn fn = tensor_map_encoder();
+  if (fn == nullptr) return false;
+  const cuuint64_t row = (cuuint64_t)g.heads * g.D * 2;
+  cuuint64_t dims[5] = {(cuuint64_t)g.D, (cuuint64_t)g.heads, (cuuint64_t)g.W, (cuuint64_t)g.H,
+                        (cuuint64_t)g.T * g.B};
+  cuuint64_t strides[4] = {(cuuint64_t)g.D * 2, row, row * g.W, row * g.W * g.H};
+  cuuint32_t box[5] = {64, 1, (cuuint32_t)g.ww, (cuuint32_t)g.wh, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D>
 cudaError_t launch_arm_d(const void* q, const void* k, const Geo& g, const Rf1Args& a, const int* coords,
                          float* partial, int32_t* status, cudaStream_t s) {
   using C = ArmCfg<D>;
   CUtensorMap tq0, tk0, tq1, tk1;
-  if (!make_sample_map(&tq0, q, g, a.S[0], 1) || !make_sample_map(&tk0, k, g, a.S[0], 1) ||
-      !make_sample_map(&tq1, q, g, a.S[1], a.omega) || !make_sample_map(&tk1, k, g, a.S[1], a.omega))
+  const bool ok0 = a.wslots ? (make_frame_window_map(&tq0, q, g) && make_frame_window_map(&tk0, k, g))
+                            : (make_sample_map(&tq0, q, g, a.S[0], 1) && make_sample_map(&tk0, k, g, a.S[0], 1));
+  if (!ok0 || !make_sample_map(&tq1, q, g, a.S[1], a.omega) || !make_sample_map(&tk1, k, g, a.S[1], a.omega))
     return cudaErrorInvalidValue;
   static int configured_device = -1;  // one flag per instance (per D)
   int dev = 0;
@@ -425,7 +470,7 @@ cudaError_t launch_rf1(const void* q, const void* k, const Geo& g, const Rf1Args
                        int32_t* cls_out, float* recall_out, int32_t* idx, int32_t* cnt, int kmax,
                        int32_t* status, cudaStream_t s) {
   const int ns = a.S[0] + a.S[1];
-  arm_coords_kernel<<<(ns + 255) / 256, 256, 0, s>>>(a, w.coords);
+  arm_coords_kernel<<<(ns + 255) / 256, 256, 0, s>>>(a, g.nbh, w.coords);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = g.D == 128 ? launch_arm_d<128>(q, k, g, a, w.coords, w.partial, status, s)

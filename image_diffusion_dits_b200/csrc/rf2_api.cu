@@ -150,8 +150,14 @@ int v1_prepare(const rf2_geom* g, const rf2_v1_params* p, unsigned flags, V1Call
   if ((long long)geo.B * geo.heads > 65535) return RF2_ERR_UNSUPPORTED;  // grid z
   rf2::Rf1Args a;
   const long long omega = p->omega == 0 ? g->T : p->omega;
-  a.S[0] = g->H * g->W;
-  a.S[1] = (int)((geo.N + omega - 1) / omega);
+  // The local sample (frame 0) goes window by window when a tile holds whole windows,
+  // so that 32 consecutive keys share a window; pad slots of partial windows are skipped.
+  const int wslots = g->wh * g->ww;
+  a.wslots = (wslots == 32 || wslots == 64 || wslots == 128) ? wslots : 0;
+  a.S_real[0] = g->H * g->W;
+  a.S[0] = a.wslots ? geo.nbh * geo.nbw * a.wslots : a.S_real[0];
+  a.S[1] = a.S_real[1] = (int)((geo.N + omega - 1) / omega);
+  a.T = g->T;
   a.coord_off[0] = 0;
   a.coord_off[1] = a.S[0];
   a.tiles_max = (max(a.S[0], a.S[1]) + 127) / 128;

@@ -123,8 +123,12 @@ inline MaskScratch mask_scratch_layout(const Geo& g, unsigned char* base) {
 // raster token).  R[p][l] is the band radius of level l = (static bandwidth, 1/8, 1/4,
 // 1/2) on that sample's axis (windows of a slab for p = 0, temporal blocks for p = 1).
 struct Rf1Args {
-  int S[2];           // samples
+  int S[2];           // sample slots (the local sample may hold pad slots, see wslots)
+  int S_real[2];      // real samples (the mean's denominator)
   int coord_off[2];   // offsets of each sample's coordinates in the coordinate table
+  int wslots;         // > 0: the local sample is ordered window by window, wslots = wh*ww
+                      // slots per window (pad slots of partial windows included)
+  int T;
   int tiles_max;      // max over p of ceil(S[p] / 128)
   int omega, HW, W, wh, ww, nbw, wt, heads;
   int R[2][4];
