@@ -25,7 +25,10 @@
 //                       32 keys in one window takes one band test.  The halves are merged
 //                       and each warp of the first half writes the sum over its rows of
 //                       inside / total.  Key coordinates come from a table built by
-//                       arm_coords_kernel.
+//                       arm_coords_kernel.  The local sample is taken window by window
+//                       (5-D boxes of frame 0, wh*ww slots per window, pad slots of
+//                       partial windows marked and skipped), so its chunks share a
+//                       window; the global sample is every omega-th token (4-D boxes).
 //   arm_finalize_kernel: per (b, head) the recall (rows summed in a fixed order), the
 //                       class and the band radius or stride.
 //   rf1_lists_kernel   : one warp per (b, head, query block): ascending kept list by
