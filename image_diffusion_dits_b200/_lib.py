@@ -39,6 +39,7 @@ EXPORTS = (
     "rf2_v1_kmax",
     "rf2_v1_workspace_size",
     "rf2_v1_predict_mask",
+    "rf2_selftest_wait_timeout",
     "rf2_status_string",
 )
 
@@ -92,6 +93,7 @@ _SIGS = {
     "rf2_v1_workspace_size": (ctypes.c_size_t, [_gp, ctypes.POINTER(Rf2V1Params), ctypes.c_uint]),
     "rf2_v1_predict_mask": (ctypes.c_int, [_vp, _vp, _gp, ctypes.POINTER(Rf2V1Params), ctypes.c_uint, _i32p,
                                            _i32p, ctypes.c_int, _i32p, _vp, _vp, ctypes.c_size_t, _vp]),
+    "rf2_selftest_wait_timeout": (ctypes.c_int, [_i32p, ctypes.c_double, ctypes.c_double, _vp]),
     "rf2_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
 

@@ -300,6 +300,15 @@ int rf2_v1_predict_mask(const void* q, const void* k, const rf2_geom* g, const r
                         unsigned flags, int32_t* idx, int32_t* cnt, int kmax, int32_t* head_class,
                         float* recall, void* ws, size_t ws_bytes, void* stream);
 
+/* rf2_selftest_wait_timeout - diagnostic of the bounded device waits of every kernel.
+ * Launches two one-warp CTAs on `stream` that each wait on an mbarrier that nothing
+ * arrives at: the first gives up after short_s seconds and writes RF2_ERR_TIMEOUT to
+ * *status (a device int32 the caller zeroes first); the second (limit long_s) gives up
+ * as soon as it sees that value.  0 < short_s <= long_s <= 5.  Returns RF2_OK once
+ * launched (the caller synchronises and reads *status), RF2_ERR_INVALID_ARG or
+ * RF2_ERR_CUDA. */
+int rf2_selftest_wait_timeout(int32_t* status, double short_s, double long_s, void* stream);
+
 /* rf2_status_string - static, human-readable text of a status code. */
 const char* rf2_status_string(int status);
 

@@ -206,3 +206,12 @@ def test_v1_rejects_bad_parameters():
     with pytest.raises(rf2.Rf2Error) as ei:
         rf2.v1_kmax(rf2.Geometry(**V1_GEOMS[0], no_permute=True))
     assert ei.value.code == _lib.RF2_ERR_UNSUPPORTED
+
+
+def test_selftest_wait_timeout_rejects_bad_arguments_without_launch():
+    lib = _lib.load()
+    assert lib.rf2_selftest_wait_timeout(None, 0.01, 0.1, None) == _lib.RF2_ERR_INVALID_ARG
+    assert lib.rf2_selftest_wait_timeout(8, 0.0, 0.1, None) == _lib.RF2_ERR_INVALID_ARG
+    assert lib.rf2_selftest_wait_timeout(8, 0.2, 0.1, None) == _lib.RF2_ERR_INVALID_ARG
+    assert lib.rf2_selftest_wait_timeout(8, 0.1, 6.0, None) == _lib.RF2_ERR_INVALID_ARG
+    assert lib.rf2_selftest_wait_timeout(6, 0.01, 0.1, None) == _lib.RF2_ERR_INVALID_ARG   # misaligned

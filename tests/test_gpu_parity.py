@@ -492,3 +492,21 @@ def test_step_attention_other_generators_and_fp8(method, fp8):
         assert same(got, ref), (method, fp8, step)
     if method == "rf1":
         assert sa.head_classes(0).shape == (g.B, g.heads)
+
+
+def test_bounded_wait_times_out_reports_and_leaves_the_context_usable():
+    """A wait on a barrier that nothing completes ends by its time limit with
+    RF2_ERR_TIMEOUT in the status word, a second CTA with a long limit gives up on seeing
+    it, and the context keeps working (a parity-checked call afterwards)."""
+    from image_diffusion_dits_b200 import _lib
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    rc = _lib.load().rf2_selftest_wait_timeout(status.data_ptr(), 0.05, 3.0, torch.cuda.current_stream().cuda_stream)
+    e1.record()
+    torch.cuda.synchronize()
+    assert rc == 0
+    assert int(status.item()) == _lib.RF2_ERR_TIMEOUT
+    elapsed = e0.elapsed_time(e1) / 1e3
+    assert 0.04 <= elapsed < 2.5, elapsed          # the long wait stopped early
+    test_attention_end_to_end("tiny")
