@@ -215,3 +215,18 @@ def test_selftest_wait_timeout_rejects_bad_arguments_without_launch():
     assert lib.rf2_selftest_wait_timeout(8, 0.2, 0.1, None) == _lib.RF2_ERR_INVALID_ARG
     assert lib.rf2_selftest_wait_timeout(8, 0.1, 6.0, None) == _lib.RF2_ERR_INVALID_ARG
     assert lib.rf2_selftest_wait_timeout(6, 0.01, 0.1, None) == _lib.RF2_ERR_INVALID_ARG   # misaligned
+
+
+def test_fp8_paths_refuse_unsupported_shapes_before_any_launch():
+    """The e4m3 attention needs D = 128 and 128-token blocks: other shapes are refused on
+    the host (no device call is made, so this runs without a GPU)."""
+    lib = _lib.load()
+    g = _g(D=64)                                     # 64-token blocks, D = 64
+    cg = g.c()
+    p = 1 << 20                                      # aligned stand-in addresses, never dereferenced
+    st = lib.rf2_sparse_attn_fp8(p, p, p, p, p, p, 4, ctypes.byref(cg), 0.0, p, 0, 0, None)
+    assert st == _lib.RF2_ERR_UNSUPPORTED
+    ws = lib.rf2_workspace_size(ctypes.byref(cg), 0.5, 1, _lib.RF2_FP8, 1)
+    assert ws > 0
+    st = lib.rf2_attention(p, p, p, ctypes.byref(cg), 0.5, 1, 0.0, p, None, p, ws, _lib.RF2_FP8, None)
+    assert st == _lib.RF2_ERR_UNSUPPORTED

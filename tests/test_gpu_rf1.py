@@ -63,6 +63,11 @@ PLANTED = [
     (dict(B=1, heads=5, T=4, H=16, W=16, D=64, wt=1, wh=8, ww=8), "tsxts", dict()),
     (dict(B=2, heads=3, T=5, H=9, W=17, D=128, wt=2, wh=8, ww=8), "sxt", dict(dynamic=True, omega=7)),
     (dict(B=1, heads=4, T=3, H=24, W=40, D=128, wt=1, wh=8, ww=8), "txst", dict(bandwidth=0.5, tau=3)),
+    # window slots per frame: 32 (wt = 2, 64-token blocks), 128, and 16 (raster-order
+    # local sample: a window's frame slice is not a whole number of 32-key chunks)
+    (dict(B=1, heads=3, T=4, H=12, W=20, D=64, wt=2, wh=4, ww=8), "tsx", dict()),
+    (dict(B=1, heads=3, T=3, H=16, W=40, D=128, wt=1, wh=8, ww=16), "stx", dict(dynamic=True)),
+    (dict(B=1, heads=3, T=8, H=12, W=12, D=64, wt=4, wh=4, ww=4), "xts", dict()),
 ]
 
 
