@@ -147,3 +147,29 @@ def test_fp8_attention_batches_and_raster_blocks(shape, no_permute):
         g_rows.append(got[b, toks, h])
         r_rows.append(ref)
     print(shape, no_permute, _close(np.concatenate(g_rows), np.concatenate(r_rows), "fp8 attention"))
+
+
+def test_fp8_empty_rows_and_bad_indices():
+    """A row with no kept block writes zeros; ids outside [0, Nb) are skipped and reported
+    (RF2_ERR_BAD_INDEX) while the valid ids of the row are still used."""
+    shape = dict(B=1, heads=1, T=2, H=16, W=16, D=128, wt=2, wh=8, ww=8)
+    g, og = rf2.Geometry(**shape), O.geom(**shape)
+    q, k, v = _bits(g, 1700)
+    q8, k8, v8, sc = rf2.quantize_fp8(to_dev(q), to_dev(k), to_dev(v), g)
+    idx = torch.tensor([[[[0, 1, 2, 3], [2, 99, -4, 3], [0, 1, 2, 3], [1, 3, 0, 2]]]], dtype=torch.int32,
+                       device="cuda")
+    cnt = torch.tensor([[[0, 4, 2, 1]]], dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = rf2.sparse_attn_fp8(q8, k8, v8, sc, idx, cnt, g, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 5
+    got = to_f64(out)
+    quant = F8.quantised_inputs(*(bf16_bits_to_f64(a) for a in (q, k, v)), og)
+    deq = [t[3] for t in quant]
+    tok = O.position_to_token(og)
+    t0 = tok[0:128]
+    assert np.all(got[0, t0[t0 >= 0], 0] == 0)
+    for i, lst in ((1, [2, 3]), (2, [0, 1]), (3, [1])):
+        ref = F8.fp8_attention_block(deq[0], deq[1], deq[2], og, 0, 0, i, lst, 1 / np.sqrt(128))
+        t = tok[i * 128:(i + 1) * 128]
+        _close(got[0, t[t >= 0], 0], ref[t >= 0], f"row {i}")

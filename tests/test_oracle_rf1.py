@@ -166,3 +166,14 @@ def test_classification_order_and_threshold():
     rec[0, 2, :, 0] = [0.79, 0.79]     # textural
     cls, _ = R1.rf1_classify(rec, g, p)
     assert cls[0].tolist() == [R1.TEMPORAL, R1.SPATIAL, R1.TEXTURAL]
+
+
+def test_kmax_matches_hand_worked_counts():
+    """Grid 4x4x4, windows (1, 2, 2): nbt = 4, P = 4 windows per slab.  Static 1/4: a
+    temporal row keeps 4 slabs x (windows within 1) <= 4 x 3 = 12, a spatial row
+    (slabs within 1) x 4 <= 3 x 4 = 12, textural tau 2 keeps 4 x 2 = 8: kmax 12.  With
+    RainFusion+ the widest level 1/2 gives radius 2: 4 x 4 = 16 either way."""
+    g = _g(4, 4, 4, 1, 2, 2)
+    assert R1.rf1_kmax(g, R1.Rf1Params()) == 12
+    assert R1.rf1_kmax(g, R1.Rf1Params(dynamic=True)) == 16
+    assert R1.rf1_kmax(g, R1.Rf1Params(bandwidth=0.125, tau=3)) == 4   # radius 0: 4 slabs x 1, 1 x 4; tau 3: 4 x 1
