@@ -230,3 +230,10 @@ def test_fp8_paths_refuse_unsupported_shapes_before_any_launch():
     assert ws > 0
     st = lib.rf2_attention(p, p, p, ctypes.byref(cg), 0.5, 1, 0.0, p, None, p, ws, _lib.RF2_FP8, None)
     assert st == _lib.RF2_ERR_UNSUPPORTED
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    """No CPU fallback: loading the library from a path without it raises."""
+    monkeypatch.setattr(_lib, "_lib", None)
+    with pytest.raises(ImportError):
+        _lib.load(str(tmp_path / "librf2.so"))
