@@ -237,3 +237,36 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(_lib, "_lib", None)
     with pytest.raises(ImportError):
         _lib.load(str(tmp_path / "librf2.so"))
+
+
+from hypothesis import given, settings, strategies as st   # noqa: E402
+
+
+_WINDOWS = [(1, 8, 8), (2, 8, 8), (1, 8, 16), (2, 4, 8), (1, 4, 16), (4, 4, 4), (2, 4, 16)]
+
+
+@settings(max_examples=60, deadline=None)
+@given(T=st.integers(1, 9), H=st.integers(1, 40), W=st.integers(1, 40), win=st.sampled_from(_WINDOWS),
+       bw=st.sampled_from([0.05, 0.125, 0.25, 0.3, 0.5, 0.75, 1.0]), tau=st.integers(1, 5), dyn=st.booleans())
+def test_v1_kmax_random_geometries_match_oracle(T, H, W, win, bw, tau, dyn):
+    wt, wh, ww = win
+    geo = dict(B=1, heads=1, T=T, H=H, W=W, D=64, wt=wt, wh=wh, ww=ww)
+    og = O.geom(**geo)
+    if og.Nb > 1024:
+        return
+    prm = dict(bandwidth=bw, tau=tau, dynamic=dyn)
+    assert rf2.v1_kmax(rf2.Geometry(**geo), rf2.V1Params(**prm)) == O.rf1.rf1_kmax(og, O.rf1.Rf1Params(**prm))
+
+
+@settings(max_examples=60, deadline=None)
+@given(T=st.integers(1, 9), H=st.integers(1, 40), W=st.integers(1, 40), win=st.sampled_from(_WINDOWS),
+       s=st.floats(0.0, 1.0), sink=st.booleans(), additive=st.booleans(), flat=st.booleans())
+def test_kept_count_random_geometries_match_oracle(T, H, W, win, s, sink, additive, flat):
+    wt, wh, ww = win
+    geo = dict(B=1, heads=1, T=T, H=H, W=W, D=64, wt=wt, wh=wh, ww=ww)
+    og = O.geom(**geo, no_permute=flat)
+    if og.Nb > 1024:
+        return
+    g = rf2.Geometry(**geo, no_permute=flat)
+    assert (g.Nb, g.Npad) == (og.Nb, og.Npad)
+    assert rf2.kept_count(g, s, sink, additive) == O.kept_count(og, s, sink, additive)
