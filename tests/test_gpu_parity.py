@@ -510,3 +510,35 @@ def test_bounded_wait_times_out_reports_and_leaves_the_context_usable():
     elapsed = e0.elapsed_time(e1) / 1e3
     assert 0.04 <= elapsed < 2.5, elapsed          # the long wait stopped early
     test_attention_end_to_end("tiny")
+
+
+def test_attention_captures_in_a_cuda_graph():
+    """The fused call allocates nothing and never synchronises, so it can be captured in a
+    CUDA graph: a replay reproduces the eager result bit for bit, and a replay after new
+    inputs are copied into the captured buffers gives the new inputs' result."""
+    wl, g, og = _geoms("video480p")
+    q, k, v = (to_dev(a) for a in _inputs("video480p"))
+    ws = torch.empty(rf2.workspace_size(g, wl.sparsity, wl.sink), dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(q)
+    rf2.attention(q, k, v, g, wl.sparsity, wl.sink, ws=ws, out=out)        # eager, also first-use setup
+    torch.cuda.synchronize()
+    ref = out.clone()
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            rf2.attention(q, k, v, g, wl.sparsity, wl.sink, ws=ws, out=out)
+    torch.cuda.current_stream().wait_stream(side)
+    out.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    q2, k2, v2 = (to_dev(a) for a in _rand_bits(g, 4242))
+    for dst, src in ((q, q2), (k, k2), (v, v2)):
+        dst.copy_(src)
+    graph.replay()
+    torch.cuda.synchronize()
+    ref2 = rf2.attention(q2, k2, v2, g, wl.sparsity, wl.sink)
+    assert torch.equal(out.view(torch.int16), ref2.view(torch.int16))
+    del graph
