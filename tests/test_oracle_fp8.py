@@ -4,7 +4,6 @@ the per-block quantisation.  CPU only."""
 import os
 
 import numpy as np
-import pytest
 import torch
 
 import oracle as O
