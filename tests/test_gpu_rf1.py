@@ -1,7 +1,9 @@
 """GPU parity of the RainFusion v1 mask generators (ARM recall on the tensor cores, head
 classes, RainFusion+ bandwidth, kept lists) against the fp64 oracle, and the attention
 they drive.  Recall within 2e-4; classes equal wherever the oracle's recall is not within
-1e-3 of a threshold it is compared with; kept lists and counts bit-exact for those heads."""
+1e-3 of a threshold it is compared with; kept lists and counts bit-exact for those heads.
+The class is also decided by the oracle from the kernel's own fp32 recalls (thresholds as
+fp32 values): that decision, and its lists, must equal the kernel's on every head."""
 import numpy as np
 import pytest
 import torch
@@ -43,6 +45,21 @@ def _check(q, k, g, og, p, heads=None):
     assert err <= RECALL_TOL, f"recall differs by {err:.2e}"
     ref_cls, ref_prm = R1.rf1_classify(ref_rec, og_h, op)
     dec = _decided(ref_rec, op)
+    # The class is an integer decided from floating point: decided again by the oracle
+    # from the kernel's own fp32 recalls against the thresholds as fp32 values, it must
+    # match the kernel's class and lists on every head, near a threshold or not.
+    op32 = R1.Rf1Params(**{**{f: getattr(op, f) for f in ("bandwidth", "tau", "omega", "dynamic")},
+                           "alpha": float(np.float32(op.alpha)), "recall_target": float(np.float32(op.recall_target))})
+    k_cls, k_prm = R1.rf1_classify(got_rec, og_h, op32)
+    assert np.array_equal(cls.cpu().numpy()[:, hs], k_cls)
+    k_lists = R1.rf1_lists(og_h, k_cls, k_prm)
+    all_idx, all_cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    for b in range(og.B):
+        for hi, h in enumerate(hs):
+            for i in range(og.Nb):
+                want = k_lists[b][hi][i]
+                assert all_idx[b, h, i, :len(want)].tolist() == want.tolist()
+                assert int(all_cnt[b, h, i]) == len(want)
     gcls = cls.cpu().numpy()[:, hs]
     assert np.all(gcls[dec] == ref_cls[dec])
     lists = R1.rf1_lists(og_h, ref_cls, ref_prm)
