@@ -1,8 +1,9 @@
 // e4m3 variant of the block-sparse attention, sm_100a (tcgen05 kind::f8f6f4 + TMEM + TMA).
 //
 // The block-sparse attention of RainFusion2.0 (mlsanity index page: title, Abstract) with
-// its operands quantised to FP8, as the pages suggest combining the method with other
-// acceleration.  Q, K and V carry one e4m3 scale per (batch, head, block):
+// its operands quantised to FP8, following the sciencestack page's TL;DR, which points to
+// integrating quantisation for further speed.  Q, K and V carry one e4m3 scale per
+// (batch, head, block):
 //   quant_fp8_kernel : per block, amax over its real tokens and the head's D channels,
 //                      inv = 448 / amax and scale = amax / 448 (fp32, rounded), codes =
 //                      e4m3(x * inv) (round to nearest even, saturating).  Reads the

@@ -193,8 +193,9 @@ int rf2_attention(const void* q, const void* k, const void* v, const rf2_geom* g
                   double sparsity, int sink, float scale, void* o, int32_t* idx_out,
                   void* ws, size_t ws_bytes, unsigned flags, void* stream);
 
-/* e4m3 variant of the attention.  The pages suggest combining the block-sparse attention
- * with quantisation; the FP8 form below is this library's reading.  Every (batch, head,
+/* e4m3 variant of the attention.  The sciencestack page's TL;DR points to integrating
+ * quantisation with the block-sparse attention for further speed; the FP8 form below is
+ * this library's reading.  Every (batch, head,
  * block) of Q, K and V gets one scale: amax = max |x| over the block's real tokens and
  * the head's D channels, inv = 448 / amax, scale = amax / 448 (fp32, rounded to
  * nearest; amax = 0 gives 0 for both); code = e4m3(x * inv) with round to nearest even

@@ -4,9 +4,9 @@ TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the 
 baseline leg of ``bench.py`` may import this module.  It shares no code with the CUDA
 library.
 
-The pages suggest combining the block-sparse attention with quantisation (RF2 index
-page, Abstract: the framework is "hardware-efficient" and compatible with other
-acceleration; the FP8 form is this build's reading, not a method the pages specify).
+The pages point to pairing the block-sparse attention with quantisation for further
+speed (RF2 sciencestack page, TL;DR, its closing remark on integration with quantisation
+or distillation); the FP8 form is this build's reading, not a method the pages specify.
 Reading used here:
   - Q, K and V are each quantised to e4m3 with one scale per (batch, head, block), the
     block being the same 3D window (or raster block) the mask works on;
