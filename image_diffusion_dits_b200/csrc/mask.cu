@@ -1,6 +1,6 @@
-// Online mask prediction (RainFusion2.0, mlsanity index page, Abstract, insight (1)
-// "block-wise mean values as representative tokens for sparse mask prediction" and
-// insight (3) "first-frame sink"; sciencestack page, TL;DR "online adaptive").
+// Online mask prediction (RainFusion2.0, mlsanity index page, Abstract, insight (1): the
+// mean of each block stands in for its tokens when the mask is predicted; insight (3):
+// the first-frame sink; sciencestack page, TL;DR: the mask is predicted online, per call).
 //
 //   pool   : qbar/kbar[b, head, j, :] = fp32 mean of the real tokens of block j.
 //            HBM-bound streaming reduction over the permuted Q and K.
@@ -8,7 +8,8 @@
 //            split into three bf16 parts (hi + mid + lo, about 24 significant bits) and
 //            the six products that matter at fp32 precision are accumulated in fp32.
 //   topk   : per row, the sink blocks plus the m best other blocks (ties to the lower
-//            id) as an ascending list; one warp per row, exact bitwise search.
+//            id) as an ascending list; one warp per row, a bracketed search for the cut
+//            (interpolation and bisection steps in turn) that ends on the exact m-th key.
 #include "rf2_common.cuh"
 #include "sm100_ptx.cuh"
 

@@ -31,20 +31,61 @@ static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
 // Device address of g_scratch per device.  In host code the name g_scratch is only a
 // host-side stand-in; a kernel given it would fault, or read host memory where the GPU
-// can reach it.  The address is looked up once per device, with that device current.
-void* g_scratch_addr[kMaxDevices] = {nullptr};
+// can reach it.  The address is looked up with the device current and kept together with
+// the id of the context it belongs to: after a cudaDeviceReset the device gets a new
+// primary context (with a new id) in which the module, and the array, are loaded anew,
+// so the address is looked up again instead of reusing a stale one.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+struct ScratchSlot {
+  unsigned long long ctx_id;  // 0: not looked up yet
+  void* addr;
+};
+ScratchSlot g_scratch_slot[kMaxDevices] = {};
 std::mutex g_scratch_mutex;
+
+// Id of the calling thread's current context (never 0), or 0 if the driver cannot say.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+    looked_up = true;
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id + 1;  // context ids may start at 0; 0 here means "unknown"
+}
 
 int scratch_for_current_device(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RF2_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
+  // cudaFree(nullptr) is the runtime's documented way to make the device's primary
+  // context current (it frees nothing), so that the id below is the context the kernels
+  // of this call will run in.
+  if (cudaFree(nullptr) != cudaSuccess) return RF2_ERR_CUDA;
+  const unsigned long long ctx = current_context_id();
+  ScratchSlot& slot = g_scratch_slot[dev];
+  if (slot.addr == nullptr || ctx == 0 || slot.ctx_id != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return RF2_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+    slot.addr = p;
+    slot.ctx_id = ctx;
   }
-  *out = g_scratch_addr[dev];
+  *out = slot.addr;
   return RF2_OK;
 }
 

@@ -8,8 +8,8 @@
  * (batch, head, query block), the key blocks to keep at a target sparsity, a first-frame
  * sink that always keeps the key blocks of the first temporal window, attention over the
  * kept blocks only, and the inverse permutation.  Passages that define each step are
- * cited per entry point below (mlsanity index page, Abstract, "key technical insights"
- * (1)-(3); sciencestack page, TL;DR and Figures 1-3).  The pages give no formulas; the
+ * cited per entry point below (mlsanity index page, Abstract, the three key technical
+ * insights (1)-(3); sciencestack page, TL;DR and Figures 1-3).  The pages give no formulas; the
  * readings used here are stated with each call.
  *
  * Conventions (every entry point):
@@ -81,9 +81,9 @@ enum rf2_flags {
     RF2_FP8 = 16u
 };
 
-/* rf2_permute - 3D window permutation (mlsanity index page, Abstract, insight (2)
- * "spatiotemporal-aware token permutation"; sciencestack page, TL;DR "3D window
- * permutation" and Figure 3).
+/* rf2_permute - 3D window permutation (mlsanity index page, Abstract, insight (2): tokens
+ * are reordered so that each block is a spatio-temporal window; sciencestack page, TL;DR
+ * and Figure 3).
  *   x  : [B, N, heads, D] bf16, raster order (read).
  *   xp : [B, Npad, heads, D] bf16 (written).  Token (t,h,w) goes to position
  *        block*blk + ((t%wt)*wh + h%wh)*ww + w%ww, block = ((t/wt)*(Hp/wh) + h/wh)*(Wp/ww)
@@ -111,8 +111,8 @@ size_t rf2_workspace_size(const rf2_geom* g, double sparsity, int sink, unsigned
                           int attention);
 
 /* rf2_predict_mask - online mask prediction on permuted Q and K (mlsanity index page,
- * Abstract, insight (1) "block-wise mean values as representative tokens for sparse mask
- * prediction" and insight (3) "first-frame sink").
+ * Abstract, insight (1): block means stand in for the tokens when the mask is predicted;
+ * insight (3): the first-frame sink).
  *   qp, kp : [B, Npad, heads, D] bf16, window order (read).  Pad positions are ignored.
  *            With RF2_RASTER: [B, N, heads, D], model order.
  *   Steps: qbar_i, kbar_j = fp32 mean over the real tokens of each block, per head;

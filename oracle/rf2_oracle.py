@@ -42,6 +42,7 @@ so the method's outputs beyond these pins are "parity unpinned by the pages".
 """
 from __future__ import annotations
 
+import dataclasses
 import functools
 import math
 from dataclasses import dataclass
@@ -243,13 +244,16 @@ class Selection:
     idx: np.ndarray        # int32 [B, heads, Nb, kept], ascending per row
     near_cut: List[set]    # per flattened row: block ids within the near-cut window
     kept: int
+    # per flattened row: block ids within 1e-4 * |c| of the cut alone (no floor); a
+    # subset of near_cut, kept so that rows excused only by the floor can be reported
+    near_cut_strict: List[set] = dataclasses.field(default_factory=list)
 
 
 def select_blocks(s: np.ndarray, g: Geom, sparsity: float, sink: bool,
                   sink_additive: bool = False, near_rel: float = 1e-4) -> Selection:
     """Per (b, head, query block) row: the sink blocks plus the top-m other valid blocks
     by pooled score, ties to the lower block id, list ascending (RF2 abstract, insights
-    (1) and (3); TL;DR 'online adaptive').
+    (1) and (3); TL;DR: predicted online for every call).
 
     near_cut[row] holds the non-sink valid blocks whose score lies within
     near_rel * max(|c|, 1e-2 * max_j |s_ij|) of the cut c, the midpoint between the lowest
@@ -263,6 +267,7 @@ def select_blocks(s: np.ndarray, g: Geom, sparsity: float, sink: bool,
     m = kept - len(sinks)
     idx = np.empty((B, Hh, Nq, kept), dtype=np.int32)
     near: List[set] = []
+    near_strict: List[set] = []
     sink_arr = np.array(sorted(sinks), dtype=np.int64)
     for b in range(B):
         for h in range(Hh):
@@ -274,14 +279,16 @@ def select_blocks(s: np.ndarray, g: Geom, sparsity: float, sink: bool,
                 chosen = cand[order[:m]]
                 full = np.sort(np.concatenate([sink_arr, chosen]))
                 idx[b, h, i] = full
-                ns = set()
+                ns, ns_strict = set(), set()
                 if 0 < m < len(cand):
                     # the cut lies between the lowest kept and the highest dropped score
                     cut = 0.5 * (sc[order[m - 1]] + sc[order[m]])
                     tol = near_rel * max(abs(cut), 1e-2 * float(np.max(np.abs(row))))
                     ns = set(cand[np.abs(sc - cut) <= tol].tolist())
+                    ns_strict = set(cand[np.abs(sc - cut) <= near_rel * abs(cut)].tolist())
                 near.append(ns)
-    return Selection(idx=idx, near_cut=near, kept=kept)
+                near_strict.append(ns_strict)
+    return Selection(idx=idx, near_cut=near, kept=kept, near_cut_strict=near_strict)
 
 
 def predict_mask(qp: np.ndarray, kp: np.ndarray, g: Geom, sparsity: float, sink: bool,
@@ -304,8 +311,8 @@ def _softmax_rows(z: np.ndarray) -> np.ndarray:
 def attention_block(qp: np.ndarray, kp: np.ndarray, vp: np.ndarray, g: Geom, b: int, h: int,
                     i: int, kept_ids: Sequence[int], scale: float) -> np.ndarray:
     """Output rows [blk, D] (fp64) of query block i of (b, h), attending to the tokens of
-    the kept key blocks only; pad keys are excluded (block-wise sparse attention, RF2
-    title and abstract 'skipping computations for insignificant tokens')."""
+    the kept key blocks only; pad keys are excluded (block-wise sparse attention: RF2
+    index page, title, and Abstract, where the work on unimportant tokens is skipped)."""
     blk = g.blk
     valid = position_valid(g)
     q = np.asarray(qp[b, i * blk:(i + 1) * blk, h], dtype=np.float64)

@@ -37,14 +37,17 @@ def assert_close(got: np.ndarray, ref: np.ndarray, what: str = "") -> dict:
 
 def compare_lists(gpu_idx: np.ndarray, gpu_cnt: np.ndarray, sel: "O.Selection") -> dict:
     """Bit-exact comparison of kept lists outside the near-cut window of each row.
-    Returns counts of rows that matched exactly and rows that differed only near the cut."""
+    Returns counts of rows that matched exactly, rows that differed only near the cut, and
+    among those the rows that the 1e-4 * |cut| window alone would not excuse (excused only
+    by the window's floor for cuts near zero)."""
     kept = sel.kept
     flat_o = sel.idx.reshape(-1, kept)
     flat_g = gpu_idx.reshape(len(flat_o), -1)
     cnt = gpu_cnt.reshape(-1)
     assert np.all(cnt == kept), "kept counts differ"
     assert np.all(flat_g[:, kept:] == -1), "entries after the kept count must be -1"
-    exact, near_rows, near_blocks = 0, 0, 0
+    exact, near_rows, near_blocks, floor_rows = 0, 0, 0, 0
+    strict = sel.near_cut_strict if sel.near_cut_strict else sel.near_cut
     for r in range(len(flat_o)):
         a = flat_g[r, :kept]
         b = flat_o[r]
@@ -56,4 +59,6 @@ def compare_lists(gpu_idx: np.ndarray, gpu_cnt: np.ndarray, sel: "O.Selection") 
         assert diff <= sel.near_cut[r], f"row {r}: lists differ outside the near-cut window: {sorted(diff)}"
         near_rows += 1
         near_blocks += len(diff) // 2
-    return {"rows": len(flat_o), "exact": exact, "near_cut_rows": near_rows, "near_cut_swaps": near_blocks}
+        floor_rows += 0 if diff <= strict[r] else 1
+    return {"rows": len(flat_o), "exact": exact, "near_cut_rows": near_rows, "near_cut_swaps": near_blocks,
+            "floor_only_rows": floor_rows}

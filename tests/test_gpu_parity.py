@@ -188,16 +188,22 @@ def test_attention_end_to_end_additive_sink():
     got = to_f64(out)
     tok = O.position_to_token(og)
     got_rows, ref_rows = [], []
+    sampled = near = 0
     for h in range(og.heads):
         for i in range(0, og.Nb, 7):
-            if not np.array_equal(gidx[0, h, i], sel.idx[0, h, i]):
-                continue
-            ref = O.attention_block(qf, kf, vf, og, 0, h, i, sel.idx[0, h, i], 1 / np.sqrt(og.D))
+            # a row whose list differs near the cut (already checked above) is compared
+            # with the oracle's attention over the list the kernel used
+            lst = gidx[0, h, i]
+            near += 0 if np.array_equal(lst, sel.idx[0, h, i]) else 1
+            ref = O.attention_block(qf, kf, vf, og, 0, h, i, lst, 1 / np.sqrt(og.D))
             t = tok[i * og.blk:(i + 1) * og.blk]
             keep = t >= 0
             ref_rows.append(ref[keep])
             got_rows.append(got[0, t[keep], h])
-    print("video480p additive", assert_close(np.concatenate(got_rows), np.concatenate(ref_rows), "additive"))
+            sampled += 1
+    assert sampled == og.heads * len(range(0, og.Nb, 7)) and sampled > 0
+    print("video480p additive", {"rows": sampled, "near_cut_rows": near},
+          assert_close(np.concatenate(got_rows), np.concatenate(ref_rows), "additive"))
 
 
 def test_sparse_attn_zero_sparsity_is_dense_attention():
@@ -275,16 +281,22 @@ def test_attention_end_to_end(name):
     blocks = range(og.Nb) if og.heads * og.Nb <= 2000 else rng.choice(og.Nb, 12, replace=False)
     tok = O.position_to_token(og)
     got_rows, ref_rows = [], []
+    sampled = near = 0
     for h in heads:
         for i in blocks:
-            if not np.array_equal(gidx[0, h, i], sel.idx[0, h, i]):
-                continue  # near-cut difference in the kept set: not comparable
-            ref = O.attention_block(qf, kf, vf, og, 0, h, i, sel.idx[0, h, i], 1 / np.sqrt(og.D))
+            # a row whose list differs near the cut (compare_lists checked that it differs
+            # only there) is compared with the oracle's attention over the kernel's list
+            lst = gidx[0, h, i]
+            near += 0 if np.array_equal(lst, sel.idx[0, h, i]) else 1
+            ref = O.attention_block(qf, kf, vf, og, 0, h, i, lst, 1 / np.sqrt(og.D))
             t = tok[i * og.blk:(i + 1) * og.blk]
             keep = t >= 0
             ref_rows.append(ref[keep])
             got_rows.append(got[0, t[keep], h])
-    print(name, stats, assert_close(np.concatenate(got_rows), np.concatenate(ref_rows), name))
+            sampled += 1
+    assert sampled == len(heads) * len(blocks) and sampled > 0
+    print(name, stats, {"rows_compared": sampled, "near_cut_rows": near},
+          assert_close(np.concatenate(got_rows), np.concatenate(ref_rows), name))
     del pos
 
 
@@ -376,6 +388,40 @@ def test_step_attention_follows_its_schedule():
         assert torch.equal(idx, i1) and torch.equal(cnt, c1)   # the lists of that layer's predict step
     with pytest.raises(RuntimeError):
         rf2.StepAttention(g, 0.5, wl.sink, schedule=sched)(0, 2, *inputs[0, 2])               # reuse before predict
+
+
+def test_step_attention_at_720p_shape_against_the_oracle():
+    """StepAttention's dense and predict steps compared with the oracle directly (not with
+    other CUDA calls): the Wan-720p grid, windows and head dim with 4 heads.  The predict
+    step's lists must equal the oracle's outside the near-cut window and its output the
+    oracle's attention over those lists; the dense step's output the oracle's attention
+    over every block, on sampled query blocks including partial windows."""
+    wl = WORKLOADS["wan720p"]
+    shape = dict(wl.geom(), heads=4)
+    g, og = rf2.Geometry(**shape), O.geom(**shape)
+    q, k, v = (gen_tensor(og.B, og.T, og.H, og.W, og.heads, og.D, 8100 + i) for i in range(3))
+    qd, kd, vd = (to_dev(a) for a in (q, k, v))
+    sa = rf2.StepAttention(g, wl.sparsity, wl.sink, schedule=rf2.Schedule(total_steps=10, dense_fraction=0.1))
+    o_dense = to_f64(sa(0, 0, qd, kd, vd))
+    o_pred = to_f64(sa(0, 1, qd, kd, vd))
+    idx, cnt = sa.lists(0)
+    qf, kf, vf = (bf16_bits_to_f64(O.permute(a, og)) for a in (q, k, v))
+    sel = O.predict_mask(qf, kf, og, wl.sparsity, wl.sink)
+    gidx = idx.cpu().numpy()
+    print("720p-shape predict step lists", compare_lists(gidx, cnt.cpu().numpy(), sel))
+    tok = O.position_to_token(og)
+    blocks = [0, og.nbw - 1, og.Nb // 2, og.Nb - og.nbw, og.Nb - 1]   # first, partial w, middle, partial t/h
+    for what, out, lists in (("dense", o_dense, None), ("predict", o_pred, gidx)):
+        got_rows, ref_rows = [], []
+        for h in range(og.heads):
+            for i in blocks:
+                lst = np.arange(og.Nb) if lists is None else lists[0, h, i]
+                ref = O.attention_block(qf, kf, vf, og, 0, h, i, lst, 1 / np.sqrt(og.D))
+                t = tok[i * og.blk:(i + 1) * og.blk]
+                keep = t >= 0
+                ref_rows.append(ref[keep])
+                got_rows.append(out[0, t[keep], h])
+        print("720p-shape", what, assert_close(np.concatenate(got_rows), np.concatenate(ref_rows), what))
 
 
 # ----------------------------------------------------------------------------- no-permute ablation

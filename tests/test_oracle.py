@@ -214,6 +214,21 @@ def test_near_cut_window_contains_ties_at_the_cut():
     sel = O.select_blocks(s, g, 0.25, True)  # K = 3 -> one of blocks 2, 3
     assert list(sel.idx[0, 0, 0]) == [0, 1, 3]
     assert sel.near_cut[0] == {2, 3}
+    assert sel.near_cut_strict[0] == {2, 3}
+
+
+def test_near_cut_floor_is_reported_apart_from_the_strict_window():
+    # Cut near zero relative to the row's largest score: the strict window (1e-4 * |c|)
+    # is far narrower than the floor (1e-4 * 1e-2 * max|s|).  Blocks 4 and 5 straddle the
+    # cut c = 0 (scores +-1e-7); block 3 (score 5e-7) lies inside the floor
+    # 1e-4 * 1e-2 * 100 = 1e-4 but outside the strict window of 1e-4 * |c| = 0.
+    g = _g(B=1, heads=1, T=1, H=4, W=24, D=4, wt=1, wh=4, ww=4)  # Nb = 6, sink 6 (T = 1)
+    row = np.array([100.0, 50.0, 20.0, 5e-7, 1e-7, -1e-7])
+    s = np.repeat(row.reshape(1, 1, 1, 6), g.Nb, axis=2)
+    sel = O.select_blocks(s, g, 1.0 - 5.0 / 6.0, False)  # K = 5: block 5 dropped
+    assert list(sel.idx[0, 0, 0]) == [0, 1, 2, 3, 4]
+    assert sel.near_cut[0] == {3, 4, 5}
+    assert sel.near_cut_strict[0] == set()  # |c| = 0: the strict window is empty
 
 
 # ----------------------------------------------------------------------------- attention
