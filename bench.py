@@ -23,7 +23,6 @@ import hashlib
 import json
 import math
 import os
-import re
 import statistics
 import subprocess
 import sys
@@ -47,6 +46,7 @@ def _args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-variants", action="store_true",
                    help="skip the untimed-for-the-metric variant legs (no-permute ablation, RainFusion v1)")
+    p.add_argument("--no-configs", action="store_true", help="skip the other workloads of the table")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--heads", type=int, default=None,
                    help="override the head count (smaller captures for profiling)")
@@ -74,18 +74,18 @@ def _geometry_numbers(g, kept):
     return dense, kept_flop, mask_bytes, permute_bytes, unpermute_bytes
 
 
-def _traffic_from_profile(kernel_src_sha):
-    """DRAM bytes per launch of the attention kernel from the committed ncu summary, if
-    it was taken on the current kernel source."""
-    path = os.path.join(ROOT, "profiles", "sparse_attn_wan720p.md")
-    if not os.path.exists(path):
+# DRAM traffic of one sparse_attn_kernel launch on the wan720p-shaped call, from ncu
+# (dram__bytes_read.sum + dram__bytes_write.sum) on an 8-head slice of the call, scaled by
+# 40 / 8 (every head is an independent set of CTAs, so traffic grows with the head count),
+# valid only while the kernel source has the hash below; null otherwise.
+NCU_ATTN_TRAFFIC = {"kernel_source_sha": None, "bytes_per_launch": None,
+                    "how": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum on an 8-head slice, x5"}
+
+
+def _attn_traffic(kernel_src_sha):
+    if NCU_ATTN_TRAFFIC["kernel_source_sha"] != kernel_src_sha:
         return None
-    txt = open(path).read()
-    m_sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", txt)
-    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
-    if not m_sha or not m_b or m_sha.group(1) != kernel_src_sha:
-        return None
-    return float(m_b.group(1))
+    return NCU_ATTN_TRAFFIC["bytes_per_launch"]
 
 
 def kernel_source_sha():
@@ -161,9 +161,9 @@ def job_throughput(flop_per_call, world, ms_per_call):
 
 
 def run_cpu_baseline(wl, sparsity, seconds, rows_cap=64):
-    """The fp64 oracle on a bounded sample of the same call: its mask stage on the full
-    call is skipped (attention dominates); attention is timed on sampled (head, query
-    block) rows and scaled to the full call."""
+    """The fp64 oracle on a bounded sample of the call, on inputs it generates itself (the
+    reference arm, which has no GPU results): one head's mask stage, then attention of
+    sampled query blocks of that head, scaled to the full call."""
     import numpy as np
     import torch
 
@@ -196,6 +196,136 @@ def run_cpu_baseline(wl, sparsity, seconds, rows_cap=64):
     call_s = (per_row * og.Nb + t_mask_head) * og.heads * og.B
     return {"call_s": call_s, "cores": cores, "rows": done, "per_row_s": per_row,
             "mask_head_s": t_mask_head}
+
+
+def run_cpu_baseline_and_parity(wl, sparsity, q, k, v, idx, o, seconds, attn_heads=4):
+    """The fp64 oracle on the very inputs of the timed GPU step (copied back to the host),
+    timed on the host cores, and the parity of the step's results against it:
+      - mask stage (pool, pooled scores, sink + top-k) on every head of the call, timed in
+        full; the GPU's kept lists are compared with the oracle's on every row (exact rows,
+        rows that differ only inside the near-cut window, rows excused only by that
+        window's floor, rows that differ elsewhere);
+      - attention on `attn_heads` sampled heads, a time-bounded sample of query blocks on
+        each (the first and last block and a partial window among them), timed and scaled
+        linearly to all heads and query blocks (labelled extrapolated); the GPU's output
+        rows are compared with the oracle's attention over the list the kernel used.
+    B = 1 workloads only (the configurations all have B = 1)."""
+    import numpy as np
+    import torch
+
+    import oracle as O
+    from rf2_inputs import bf16_bits_to_f64
+
+    assert wl.B == 1
+    cores = len(os.sched_getaffinity(0))
+    torch.set_num_threads(cores)
+    og = O.geom(**wl.geom())
+    one = dict(wl.geom())
+    one["heads"] = 1
+    g1 = O.geom(**one)
+    sc = 1.0 / math.sqrt(wl.D)
+    bits = lambda t: t.detach().view(torch.int16).cpu().numpy().view(np.uint16)
+    qb, kb, vb, ob = bits(q), bits(k), bits(v), bits(o)
+    gidx = idx.cpu().numpy()
+    kept = gidx.shape[-1]
+    lists = {"rows": 0, "exact": 0, "near_cut_rows": 0, "floor_only_rows": 0, "mismatch_rows": 0}
+    t_mask = 0.0
+    sels = {}
+    rng = np.random.default_rng(11)
+    attn_h = sorted(rng.choice(og.heads, min(attn_heads, og.heads), replace=False).tolist())
+    for h in range(og.heads):
+        qh, kh = (O.permute(bf16_bits_to_f64(a[:, :, h:h + 1]), g1) for a in (qb, kb))
+        t0 = time.perf_counter()
+        sel = O.predict_mask(qh, kh, g1, sparsity, wl.sink)
+        t_mask += time.perf_counter() - t0
+        if h in attn_h:
+            sels[h] = sel
+        for i in range(og.Nb):
+            a, b = gidx[0, h, i], sel.idx[0, 0, i]
+            lists["rows"] += 1
+            if np.array_equal(a, b):
+                lists["exact"] += 1
+                continue
+            diff = set(a.tolist()) ^ set(b.tolist())
+            if diff <= sel.near_cut[i]:
+                lists["near_cut_rows"] += 1
+                lists["floor_only_rows"] += 0 if diff <= sel.near_cut_strict[i] else 1
+            else:
+                lists["mismatch_rows"] += 1
+    tok = O.position_to_token(og)
+    per_head_budget = seconds / max(len(attn_h), 1)
+    err_sq = ref_sq = 0.0
+    max_abs = 0.0
+    rows = 0
+    t_attn = 0.0
+    for h in attn_h:
+        qh, kh, vh = (O.permute(bf16_bits_to_f64(a[:, :, h:h + 1]), g1) for a in (qb, kb, vb))
+        order = [0, og.Nb - 1, og.Nb - og.nbw] + rng.permutation(og.Nb).tolist()
+        seen = set()
+        t0 = time.perf_counter()
+        for i in order:
+            if i in seen or i < 0:
+                continue
+            if seen and time.perf_counter() - t0 > per_head_budget:
+                break
+            seen.add(i)
+            ref = O.attention_block(qh, kh, vh, g1, 0, 0, i, gidx[0, h, i], sc)
+            t = tok[i * og.blk:(i + 1) * og.blk]
+            keep = t >= 0
+            got = bf16_bits_to_f64(ob[0, t[keep], h])
+            d = got - ref[keep]
+            err_sq += float((d * d).sum())
+            ref_sq += float((ref[keep] ** 2).sum())
+            max_abs = max(max_abs, float(np.abs(d).max()))
+            rows += 1
+        t_attn += time.perf_counter() - t0
+    per_row = t_attn / max(rows, 1)
+    call_s = t_mask + per_row * og.Nb * og.heads
+    return {"call_s": call_s, "cores": cores, "mask_all_heads_s": t_mask, "attn_rows": rows,
+            "attn_heads": attn_h, "attn_per_row_s": per_row,
+            "parity": {"lists": lists, "attn_rows": rows, "attn_max_abs": max_abs,
+                       "attn_rel_l2": math.sqrt(err_sq / max(ref_sq, 1e-300)),
+                       "tolerance": {"max_abs": 2e-2, "rel_l2": 1e-2}}}
+
+
+def run_configs(rf2, dev, stream, peaks, iters, skip=()):
+    """Every other workload of the table through the same two calls as the step
+    (rf2_predict_mask + rf2_sparse_attn, model order): ms per call, kept-tile TFLOP/s and
+    its fraction of the bf16 peak, and the mask stage's GB/s and fraction of HBM; the long
+    video at every sparsity of its sweep."""
+    import torch
+
+    from rf2_inputs import WORKLOADS, gen_tensor_torch
+
+    out = {}
+    for name, wl in WORKLOADS.items():
+        if name in skip:
+            continue
+        g = rf2.Geometry(**wl.geom())
+        q, k, v = (gen_tensor_torch(g.B, g.T, g.H, g.W, g.heads, g.D, 1000 * wl.cfg + i, dev) for i in range(3))
+        o = torch.empty_like(q)
+        for sp in wl.sparsities:
+            kept = rf2.kept_count(g, sp, wl.sink)
+            dense, kept_flop, mask_bytes, _, _ = _geometry_numbers(g, kept)
+            idx = torch.empty((g.B, g.heads, g.Nb, kept), dtype=torch.int32, device=dev)
+            cnt = torch.empty((g.B, g.heads, g.Nb), dtype=torch.int32, device=dev)
+            ws = torch.empty(rf2.workspace_size(g, sp, wl.sink, attention=False), dtype=torch.uint8, device=dev)
+            t_mask, t_attn = _time_legs(stream, iters, [
+                lambda: rf2.predict_mask(q, k, g, sp, wl.sink, kmax=kept, ws=ws, out=(idx, cnt), raster=True),
+                lambda: rf2.sparse_attn(q, k, v, idx, cnt, g, out=o, raster=True)])
+            ach = kept_flop / (t_attn * 1e-3) / 1e12
+            gbs = mask_bytes / (t_mask * 1e-3) / 1e9
+            out[f"{name}@{sp:g}"] = {
+                "geometry": f"B={wl.B} heads={wl.heads} grid={wl.T}x{wl.H}x{wl.W} D={wl.D} "
+                            f"window={wl.wt}x{wl.wh}x{wl.ww} sink={wl.sink}",
+                "kept": f"{kept}/{g.Nb}", "ms_per_call": t_mask + t_attn,
+                "dense_equiv_TFLOP/s": dense / ((t_mask + t_attn) * 1e-3) / 1e12,
+                "sparse_attn_ms": t_attn, "kept_TFLOP/s": ach, "frac_bf16_burst": ach / peaks["bf16_tflops"],
+                "predict_mask_ms": t_mask, "mask_GB/s": gbs, "mask_frac_hbm": gbs / peaks["hbm_gbs"]}
+            del idx, cnt, ws
+        del q, k, v, o
+        torch.cuda.empty_cache()
+    return out
 
 
 def _time_legs(stream, iters, legs):
@@ -390,6 +520,8 @@ def main():
         torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
+    # the step's results, kept for the parity check against the oracle at the end
+    o_step, idx_step = o.clone(), idx.clone()
     total_ms = start.elapsed_time(end)
     seg_ms = [sum(seg_ev[s][i].elapsed_time(seg_ev[s][i + 1]) for s in range(a.steps)) / a.steps
               for i in range(n_seg)]
@@ -470,18 +602,27 @@ def main():
     variants = None if a.no_variants else run_variants(rf2, g, wl, sparsity, q, k, v, o, stream, dev,
                                                         iters=max(3, min(a.steps, 5)))
 
+    configs = None
+    if not a.no_configs and a.heads is None:
+        configs = run_configs(rf2, dev, stream, peaks, iters=3, skip=(wl.name,))
+
     cpu = None
+    parity = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        cb = run_cpu_baseline(wl, sparsity, a.cpu_seconds)
+        cb = run_cpu_baseline_and_parity(wl, sparsity, q, k, v, idx_step, o_step, a.cpu_seconds)
         cpu = {"value": dense / cb["call_s"] / 1e12, "unit": unit, "cores": cb["cores"], "kind": "oracle",
                "ms_per_call": cb["call_s"] * 1e3,
-               "sample": f"attention of {cb['rows']} sampled query blocks of one head (fp64 NumPy) plus that "
-                         f"head's mask stage, scaled to {wl.heads} heads x {g.Nb} query blocks"}
+               "sample": f"fp64 NumPy oracle on the step's own inputs: mask stage on all {wl.heads} heads timed in "
+                         f"full ({cb['mask_all_heads_s']:.1f} s); attention of {cb['attn_rows']} query blocks of "
+                         f"heads {cb['attn_heads']} timed ({cb['attn_per_row_s'] * 1e3:.0f} ms each) and scaled "
+                         f"to {wl.heads} heads x {g.Nb} query blocks (extrapolated)"}
+        parity = cb["parity"]
+    del o_step, idx_step
 
     attn_ms = seg_ms[1]
     achieved = kept_flop / (attn_ms * 1e-3) / 1e12
     sha = kernel_source_sha()
-    traffic = _traffic_from_profile(sha)
+    traffic = _attn_traffic(sha)
     mask_gbs = mask_bytes / (seg_ms[0] * 1e-3) / 1e9
     line = {
         "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
@@ -510,8 +651,18 @@ def main():
         "gpu_launches": launches_per_step * a.steps,
         "e2e": e2e,
         "cpu_baseline": cpu,
+        "parity_vs_oracle": parity,
+        "configs": configs,
         "variants": variants,
     }
+    if configs is not None:
+        configs = {f"{wl.name}@{sparsity:g}": {
+            "geometry": line["config"]["workload"], "kept": f"{kept}/{g.Nb}", "ms_per_call": ms_per_step,
+            "dense_equiv_TFLOP/s": value / world, "sparse_attn_ms": attn_ms, "kept_TFLOP/s": achieved,
+            "frac_bf16_burst": achieved / peaks["bf16_tflops"], "predict_mask_ms": seg_ms[0],
+            "mask_GB/s": mask_gbs, "mask_frac_hbm": mask_gbs / peaks["hbm_gbs"], "note": "the headline step"},
+            **configs}
+        line["configs"] = configs
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

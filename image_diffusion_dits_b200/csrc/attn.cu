@@ -16,9 +16,9 @@
 // Warp roles (352 threads):
 //   warps 0-3  softmax of stream 0, warps 4-7 softmax of stream 1: thread r owns query
 //              row r = TMEM lane r.  Reads the S row in one TMEM load, online softmax in
-//              the exp2 domain (fp32 max, sum and arguments; packed f16 exp2 of each pair
-//              of arguments), writes P (bf16 pairs) over the S columns, rescales its O when
-//              its running max grows by more than 2^8.
+//              the exp2 domain (fp32 max, sum, arguments and exp2), writes P (bf16 pairs)
+//              over the S columns, rescales its O when its running max grows by more than
+//              2^8.
 //   warp 8     TMA producer of Q (once) and of K_j for each kept block j (3-stage ring).
 //   warp 9     MMA issuer: S_i = Q K_i^T (SS, K-major) into the S/P buffer of stream i%2,
 //              O_{i%2} += P_i V_i (P from TMEM, V MN-major from shared memory), then
@@ -463,13 +463,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pk[BLK / 2];
 #pragma unroll
         for (int c2 = 0; c2 < BLK / 2; ++c2) {
-          // arguments of a pair in one packed FFMA (fp32), then one packed f16 exp2 on the
-          // exp2 unit: the f16 argument (11 significant bits, |x| <= 8 here) and result
-          // carry more precision than the bf16 P they become
+          // arguments of a pair in one packed FFMA (fp32), then exp2 of each in fp32 on
+          // the exp2 unit (measured: the packed f16 form costs the exp2 unit the same time
+          // per element and needs three conversions per pair on top)
           float a0, a1;
           ptx::f2split(ptx::ffma2(ptx::f2(x[2 * c2], x[2 * c2 + 1]), sc2, nm2), a0, a1);
-          float p0, p1;
-          ptx::ex2_f16x2(a0, a1, p0, p1);
+          const float p0 = ptx::ex2(a0), p1 = ptx::ex2(a1);
           ls2[c2 & 3] = ptx::fadd2(ls2[c2 & 3], ptx::f2(p0, p1));
           pk[c2] = ptx::pack_bf16(p0, p1);
         }

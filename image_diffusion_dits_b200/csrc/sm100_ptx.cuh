@@ -67,11 +67,11 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 // and only every 65536 polls the call-wide status word in global memory, so a phase that
 // completes is seen within one poll.  Gives up (returns false) when *abort is set by
 // another thread of the CTA, when the status word reports another CTA's timeout, or after
-// `limit_ns`; in the last case it raises both flags.
+// `limit_ns`; in the last case it raises both flags.  The first probe is a try_wait
+// (measured ~40 clk on a completed phase, against ~70 for a test_wait followed by it).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           volatile int* gstatus, uint64_t limit_ns,
                                           int timeout_code) {
-  if (mbar_test_wait(bar, parity)) return true;  // already complete: no suspend logic
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   uint32_t spins = 0;
@@ -389,18 +389,6 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^a0, 2^a1 on the exp2 unit in one packed f16 operation: the arguments are rounded to
-// f16 (nearest), the results widened back to fp32.  -inf gives 0; arguments below about
-// -24 underflow to 0.
-__device__ __forceinline__ void ex2_f16x2(float a0, float a1, float& p0, float& p1) {
-  uint32_t h2, e2;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h2) : "f"(a1), "f"(a0));  // first source -> upper half
-  asm("ex2.approx.f16x2 %0, %1;" : "=r"(e2) : "r"(h2));
-  asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tcvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
-      : "=f"(p0), "=f"(p1)
-      : "r"(e2));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {

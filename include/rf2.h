@@ -169,7 +169,7 @@ int rf2_predict_mask_noalloc(const void* qp, const void* kp, const rf2_geom* g,
  *   is written.
  *   scale : softmax scale, > 0; 0 means 1/sqrt(D) (negative: RF2_ERR_INVALID_ARG).
  *   Softmax statistics and the accumulator
- *   are fp32; exp2 is taken in f16 and P rounded to bf16 for the P.V product.
+ *   are fp32; exp2 is taken in fp32 and P rounded to bf16 for the P.V product.
  *   status : optional device int32 (may be NULL); when given it must be zero on entry
  *   and receives RF2_ERR_BAD_INDEX / RF2_ERR_TIMEOUT if the kernel detects one
  *   (out-of-range ids are skipped, never dereferenced).  With RF2_CHECKED and a status

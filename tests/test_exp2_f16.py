@@ -1,8 +1,8 @@
-"""Host-side bound for the attention kernel's packed f16 exp2 (sm100_ptx.cuh, ex2_f16x2).
+"""Host-side bound for the packed f16 exp2 of the e4m3 attention kernel (attn_fp8.cu).
 
-The softmax forms its exp2 arguments in fp32, with x <= 8 (the running max moves once
+Its softmax forms the exp2 arguments in fp32, with x <= 8 (the running max moves once
 a score exceeds it by 8), rounds each pair to f16 and takes 2^x of both in one f16
-operation; P is then rounded to bf16 for the P V product.  This checks, with exact
+operation; P is then rounded further for the P V product.  This checks, with exact
 exp2 in float64, that rounding the argument to f16 and the result to f16 perturbs P by
 less than the bf16 rounding of P itself, over the argument range the softmax uses,
 and that masked keys (-inf) give exactly 0.  (The hardware result is compared with the

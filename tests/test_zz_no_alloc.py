@@ -56,6 +56,17 @@ def test_noalloc_matches_predict_mask_on_consecutive_calls():
         assert int(cnt[0, 0, 0]) == kept
 
 
+def test_noalloc_checked_mode_returns_the_device_status():
+    """With RF2_CHECKED the call waits for its work and returns the device status word
+    (0 here), and its lists still equal rf2_predict_mask's."""
+    wl, g, qp, kp = _permuted("tiny")
+    kept = rf2.kept_count(g, wl.sparsity, wl.sink)
+    ref_idx, ref_cnt = rf2.predict_mask(qp, kp, g, wl.sparsity, wl.sink, kmax=kept)
+    for _ in range(2):
+        idx, cnt = _noalloc(qp, kp, g, wl.sparsity, wl.sink, _lib.RF2_CHECKED, kept)
+        assert torch.equal(idx, ref_idx) and torch.equal(cnt, ref_cnt)
+
+
 def test_noalloc_rejects_shapes_beyond_its_scratch():
     lib = _lib.load()
     wl = WORKLOADS["wan720p"]
