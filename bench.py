@@ -78,8 +78,9 @@ def _geometry_numbers(g, kept):
 # (dram__bytes_read.sum + dram__bytes_write.sum) on an 8-head slice of the call, scaled by
 # 40 / 8 (every head is an independent set of CTAs, so traffic grows with the head count),
 # valid only while the kernel source has the hash below; null otherwise.
-NCU_ATTN_TRAFFIC = {"kernel_source_sha": None, "bytes_per_launch": None,
-                    "how": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum on an 8-head slice, x5"}
+NCU_ATTN_TRAFFIC = {"kernel_source_sha": "fecc4ae4b6e445a3", "bytes_per_launch": 5 * (541.100032e6 + 166.780672e6),
+                    "how": "ncu --set full, dram__bytes_read.sum + dram__bytes_write.sum of one launch on an "
+                           "8-head slice of the call (541.1 + 166.8 MB), x5 for 40 heads"}
 
 
 def _attn_traffic(kernel_src_sha):
@@ -636,6 +637,7 @@ def main():
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                     "traffic_source": NCU_ATTN_TRAFFIC["how"] if traffic is not None else None,
                      "kernel": "sparse_attn_kernel<128,128>", "peak_source": peaks["source"] + " burst",
                      "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
                                            if peaks.get("bf16_tflops_sustained") else None),

@@ -48,6 +48,34 @@ def _rand_bits(g, seed):
 
 # ----------------------------------------------------------------------------- permutation
 
+@pytest.mark.parametrize("shape", [RAGGED[1], dict(B=1, heads=2, T=4, H=16, W=40, D=128, wt=2, wh=8, ww=8)])
+@pytest.mark.parametrize("raster", [False, True])
+def test_predict_mask_exact_ties_take_the_lowest_ids(shape, raster):
+    """Every key block of a row with the same pooled score (K constant over the grid, so
+    every block mean is that constant): the scores tie exactly, in fp64 and in the
+    kernels' fp32, and the kept set must be the sink plus the lowest non-sink ids, bit
+    for bit (the near-cut window would excuse every candidate here, so the lists are
+    compared exactly)."""
+    g, og = rf2.Geometry(**shape), O.geom(**shape)
+    q, _, _ = _rand_bits(g, 1500)
+    rng = np.random.default_rng(1501)
+    const = rng.standard_normal(g.D)
+    kf = np.broadcast_to(const, (g.B, g.N, g.heads, g.D)).astype(np.float32)
+    from rf2_inputs import f32_to_bf16_bits
+    k = f32_to_bf16_bits(np.ascontiguousarray(kf))
+    for s_, sink in ((0.5, True), (0.7, False), (0.8, True)):
+        sel = O.predict_mask(bf16_bits_to_f64(O.permute(q, og)), bf16_bits_to_f64(O.permute(k, og)), og, s_, sink)
+        if raster:
+            idx, cnt = rf2.predict_mask(to_dev(q), to_dev(k), g, s_, sink, checked=True, raster=True)
+        else:
+            idx, cnt = rf2.predict_mask(to_dev(O.permute(q, og)), to_dev(O.permute(k, og)), g, s_, sink, checked=True)
+        got = idx.cpu().numpy()
+        assert np.array_equal(got, sel.idx), (s_, sink)
+        assert np.all(cnt.cpu().numpy() == sel.kept)
+        # the sink is blocks 0 .. nsink - 1, so the lowest ids of either kind are 0 .. kept - 1
+        assert np.array_equal(got.reshape(-1, sel.kept), np.broadcast_to(np.arange(sel.kept), (got.size // sel.kept, sel.kept)))
+
+
 @pytest.mark.parametrize("shape", RAGGED)
 def test_permute_unpermute_ragged_bit_exact(shape):
     g, og = rf2.Geometry(**shape), O.geom(**shape)
