@@ -249,93 +249,41 @@ __global__ void __launch_bounds__(kSThreads) scores_kernel(const __grid_constant
 }
 
 // ------------------------------------------------------------------------------- top-k
-// Four threads per (b, head, i) row, eight rows per warp (one warp per CTA).  The warp
-// loads its rows' scores once, as order-preserving uint32 keys (every real key is > 0;
-// 0 marks a non-candidate: a sink block or a position past Nb), into shared memory.  The
-// threshold is found exactly by a bracketed search over the key range (interpolated and
-// bisection steps in turn), stopping as soon as exactly m candidates lie at or above it;
-// each count is a pass over the row in shared memory, a quarter per thread (every fourth
-// group of four keys) added up with two shuffles.  Candidates above the threshold are
-// kept, and equal ones in ascending block order until m are kept.  The list (sink blocks
-// and kept candidates) is emitted in ascending order, sixteen blocks per round, with a
-// scan over the four threads.  (One warp per row measured ~2240 warp instructions per
-// row on the 720p rows: a warp-wide reduction per count and per-lane slots of the
-// search; this layout does each count with a fraction of the instructions.)
-constexpr int kTopkRows = 8;     // rows per warp (and CTA)
-constexpr int kMaxNb = 1024;
+// One warp per (b, head, i) row.  Scores map to order-preserving uint32 keys (every real
+// key is > 0; 0 marks a non-candidate).  The threshold is found exactly by a bracketed
+// search over the key range with warp-wide counts (interpolated and bisection steps in
+// turn), stopping as soon as exactly m candidates lie at or above it; candidates above it
+// are kept, and equal ones in ascending block order until m are kept.  The output list (sink blocks and kept candidates) is
+// emitted in ascending order with ballots.
+constexpr int kTopkWarps = 8;
+constexpr int kMaxPerLane = 32;  // Nb <= 1024
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Shared-memory row stride in keys: room for whole 16-key groups, and rows 64 bytes apart
-// modulo 128 so that the two rows of each quarter-warp phase of a 16-byte load fall in
-// different banks.
-__host__ __device__ __forceinline__ int topk_stride(int Nb) { return ((Nb + 31) & ~31) + 16; }
-
-__device__ __forceinline__ int quad_sum(int v) {
-  v += __shfl_xor_sync(0xffffffffu, v, 1);
-  v += __shfl_xor_sync(0xffffffffu, v, 2);
-  return v;
-}
-
-// Exclusive prefix of v over the four threads of a quad (q = lane & 3), and the total.
-__device__ __forceinline__ int quad_excl(int v, int q, int& total) {
-  int inc = v;
-  int t = __shfl_up_sync(0xffffffffu, inc, 1, 4);
-  if (q >= 1) inc += t;
-  t = __shfl_up_sync(0xffffffffu, inc, 2, 4);
-  if (q >= 2) inc += t;
-  total = __shfl_sync(0xffffffffu, inc, 3, 4);
-  return inc - v;
-}
-
-__global__ void __launch_bounds__(32) topk_kernel(const float* __restrict__ s, int32_t* __restrict__ idx,
-                                                  int32_t* __restrict__ cnt, int Nb, long long rows, int kmax,
-                                                  int kept, int nsink) {
-  extern __shared__ uint4 topk_smem[];
-  uint32_t* keys_s = reinterpret_cast<uint32_t*>(topk_smem);
-  const int lane = threadIdx.x;
-  const int rr = lane >> 2, q = lane & 3;
-  const int stride = topk_stride(Nb);
-  const int ng = (Nb + 15) >> 4;  // groups of 16 keys (four per thread, one group per pass step)
-  const long long row0 = (long long)blockIdx.x * kTopkRows;
-  for (int r = 0; r < kTopkRows; ++r) {
-    const long long row = row0 + r;
-    uint32_t* kr = keys_s + r * stride;
-    const float* sr = s + row * Nb;
-    for (int j = lane; j < ng * 16; j += 32)
-      kr[j] = (row < rows && j < Nb && j >= nsink) ? order_key(__ldg(sr + j)) : 0u;
-  }
-  __syncwarp();
-  const long long row = row0 + rr;
-  const bool live = row < rows;
-  // this thread's keys: group g holds keys 16g + 4q .. 16g + 4q + 3
-  const uint4* mk = reinterpret_cast<const uint4*>(keys_s + rr * stride) + q;
-  uint32_t kmin = 0xffffffffu, kmx = 0u;
-  for (int g2 = 0; g2 < ng; ++g2) {
-    const uint4 v = mk[4 * g2];
-    const uint32_t e[4] = {v.x, v.y, v.z, v.w};
+template <int KPL>
+__device__ __forceinline__ int count_ge(const uint32_t (&key)[KPL], uint32_t t) {
+  int c = 0;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      if (e[c] != 0u) kmin = min(kmin, e[c]);
-      kmx = max(kmx, e[c]);
-    }
+  for (int k = 0; k < KPL; ++k) c += key[k] >= t;
+  return (int)__reduce_add_sync(0xffffffffu, (uint32_t)c);
+}
+
+template <int KPL>
+__device__ __forceinline__ void topk_row(const float* __restrict__ sr, int32_t* __restrict__ out,
+                                         int32_t* __restrict__ cnt_out, int Nb, int kmax, int kept,
+                                         int nsink, int lane) {
+  uint32_t key[KPL];
+  uint32_t kmin = 0xffffffffu, kmax_key = 0u;
+#pragma unroll
+  for (int k = 0; k < KPL; ++k) {
+    const int j = k * 32 + lane;
+    key[k] = (j < Nb && j >= nsink) ? order_key(__ldg(sr + j)) : 0u;
+    if (key[k] != 0u) kmin = min(kmin, key[k]);
+    kmax_key = max(kmax_key, key[k]);
   }
-  kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, 1));
-  kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, 2));
-  kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, 1));
-  kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, 2));
-  auto count_ge = [&](uint32_t t) -> int {
-    int c = 0;
-#pragma unroll 4
-    for (int g2 = 0; g2 < ng; ++g2) {
-      const uint4 v = mk[4 * g2];
-      c += (v.x >= t) + (v.y >= t) + (v.z >= t) + (v.w >= t);
-    }
-    return quad_sum(c);
-  };
   const int m = kept - nsink;
   const int ncand = Nb - nsink;
   uint32_t thr;       // every candidate key >= thr is kept when take_eq covers all keys == thr
@@ -349,106 +297,103 @@ __global__ void __launch_bounds__(32) topk_kernel(const float* __restrict__ s, i
     // t inside the bracket, interpolated from the two counts (keys of a smooth score
     // distribution are close to uniform locally) on even steps and the midpoint on odd
     // steps, and stops when exactly m keys are >= t.  Otherwise the bracket shrinks to
-    // one value: lo is then the m-th largest key.  The rows of a warp take different
-    // numbers of steps; a finished row's quad keeps counting (the result unused) so
-    // that the shuffles stay warp-wide.
-    uint64_t lo = kmin;
-    uint64_t hi = (uint64_t)kmx + 1u;
+    // one value: lo is then the m-th largest key.
+    uint64_t lo = __reduce_min_sync(0xffffffffu, kmin);
+    uint64_t hi = (uint64_t)__reduce_max_sync(0xffffffffu, kmax_key) + 1u;
     int c_lo = ncand, c_hi = 0;
-    bool done = !live;
+    bool exact = false;
 #pragma unroll 1
-    for (int step = 0; __any_sync(0xffffffffu, !done); ++step) {
+    for (int step = 0; hi - lo > 1; ++step) {
       const uint64_t w = hi - lo;
       uint64_t off;
       if (step & 1) {
         off = w >> 1;
       } else {
-        // fp32 is precise enough for a guess (the count decides, not the guess)
-        const float frac = __fdividef((float)(c_lo - m), (float)max(c_lo - c_hi, 1));
-        off = (uint64_t)__float2uint_rz((float)w * frac);
+        const float frac = (float)(c_lo - m) / (float)(c_lo - c_hi);
+        off = (uint64_t)((double)w * (double)frac);
       }
-      off = off < 1 ? 1 : (off + 1 > w ? (w > 1 ? w - 1 : 1) : off);
+      off = off < 1 ? 1 : (off > w - 1 ? w - 1 : off);
       const uint32_t t = (uint32_t)(lo + off);
-      const int c = count_ge(t);
-      if (!done) {
-        if (c == m) {
-          lo = t;
-          done = true;
-        } else if (c > m) {
-          lo = t;
-          c_lo = c;
-        } else {
-          hi = t;
-          c_hi = c;
-        }
-        if (hi - lo <= 1) done = true;
+      const int c = count_ge<KPL>(key, t);
+      if (c == m) {
+        lo = t;
+        exact = true;
+        break;
+      }
+      if (c > m) {
+        lo = t;
+        c_lo = c;
+      } else {
+        hi = t;
+        c_hi = c;
       }
     }
+    (void)exact;
     thr = (uint32_t)lo;
   }
   // keys above thr are kept; of the keys equal to thr, the take_eq lowest ids
   int above = 0, eqc = 0;
-  for (int g2 = 0; g2 < ng; ++g2) {
-    const uint4 v = mk[4 * g2];
-    above += (v.x > thr) + (v.y > thr) + (v.z > thr) + (v.w > thr);
-    eqc += (v.x == thr) + (v.y == thr) + (v.z == thr) + (v.w == thr);
+#pragma unroll
+  for (int k = 0; k < KPL; ++k) {
+    above += key[k] > thr;
+    eqc += key[k] == thr;
   }
-  above = quad_sum(above);
-  eqc = quad_sum(eqc);
+  above = (int)__reduce_add_sync(0xffffffffu, (uint32_t)above);
+  eqc = (int)__reduce_add_sync(0xffffffffu, (uint32_t)eqc);
   const bool all = m >= ncand;
   const bool some = m > 0 && m < ncand;
   const int take_eq = some ? m - above : 0;
-  const bool split_ties = some && take_eq != eqc;
-  int32_t* out = idx + row * kmax;
-  int pos = 0, eq_taken = 0;
-  for (int g2 = 0; g2 < ng; ++g2) {
-    const uint4 v = mk[4 * g2];
-    const uint32_t e[4] = {v.x, v.y, v.z, v.w};
-    const int j0 = 16 * g2 + 4 * q;
-    // equal keys before each of this thread's four, in ascending block order
-    int eq_here = 0;
-    if (split_ties) {
+  int pos = 0;
+  if (!some || take_eq == eqc) {
+    // every key equal to thr is kept (or none is): one ballot per 32 blocks
 #pragma unroll
-      for (int c = 0; c < 4; ++c) eq_here += (e[c] == thr && e[c] != 0u);
-    }
-    int eq_total;
-    int eq_rank = eq_taken + quad_excl(eq_here, q, eq_total);
-    eq_taken += eq_total;
-    bool take[4];
-    int ntake = 0;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int j = j0 + c;
+    for (int k = 0; k < KPL; ++k) {
+      if (k * 32 >= Nb) break;
+      const int j = k * 32 + lane;
       const bool in_range = j < Nb;
       const bool is_sink = in_range && j < nsink;
-      const bool cand = in_range && !is_sink && e[c] != 0u;
-      bool t;
-      if (!split_ties) {
-        t = is_sink || (cand && (all || (some && e[c] >= thr)));
-      } else {
-        const bool eq = cand && e[c] == thr;
-        t = is_sink || (cand && e[c] > thr) || (eq && eq_rank < take_eq);
-        eq_rank += eq ? 1 : 0;
-      }
-      take[c] = t;
-      ntake += t ? 1 : 0;
+      const bool cand = in_range && !is_sink && key[k] != 0u;
+      const bool take = is_sink || (cand && (all || (some && key[k] >= thr)));
+      const uint32_t tmask = __ballot_sync(0xffffffffu, take);
+      const int p = pos + __popc(tmask & ((1u << lane) - 1u));
+      if (take && p < kmax) out[p] = j;
+      pos += __popc(tmask);
     }
-    int total;
-    int p = pos + quad_excl(ntake, q, total);
-    if (live) {
+  } else {
+    int eq_taken = 0;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        if (take[c]) {
-          if (p < kmax) out[p] = j0 + c;
-          ++p;
-        }
+    for (int k = 0; k < KPL; ++k) {
+      if (k * 32 >= Nb) break;
+      const int j = k * 32 + lane;
+      const bool in_range = j < Nb;
+      const bool is_sink = in_range && j < nsink;
+      const bool gt = in_range && !is_sink && key[k] > thr;
+      const bool eq = in_range && !is_sink && key[k] == thr;
+      const uint32_t eqmask = __ballot_sync(0xffffffffu, eq);
+      const int eq_rank = eq_taken + __popc(eqmask & ((1u << lane) - 1u));
+      const bool take = is_sink || gt || (eq && eq_rank < take_eq);
+      eq_taken += __popc(eqmask);
+      const uint32_t tmask = __ballot_sync(0xffffffffu, take);
+      const int p = pos + __popc(tmask & ((1u << lane) - 1u));
+      if (take && p < kmax) out[p] = j;
+      pos += __popc(tmask);
     }
-    pos += total;
   }
-  if (live) {
-    for (int p = pos + q; p < kmax; p += 4) out[p] = -1;
-    if (q == 0) cnt[row] = pos;
-  }
+  for (int p = pos + lane; p < kmax; p += 32) out[p] = -1;
+  if (lane == 0) *cnt_out = pos;
+}
+
+template <int KPL>
+__global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __restrict__ s,
+                                                               int32_t* __restrict__ idx,
+                                                               int32_t* __restrict__ cnt,
+                                                               int Nb, long long rows, int kmax,
+                                                               int kept, int nsink) {
+  const int lane = threadIdx.x & 31;
+  const int w = threadIdx.x >> 5;
+  const long long row = (long long)blockIdx.x * kTopkWarps + w;
+  if (row >= rows) return;
+  topk_row<KPL>(s + row * Nb, idx + row * kmax, cnt + row, Nb, kmax, kept, nsink, lane);
 }
 
 }  // namespace
@@ -505,20 +450,29 @@ cudaError_t launch_scores(const __nv_bfloat16* q3, const __nv_bfloat16* k3, floa
 
 cudaError_t launch_topk(const float* scores, int32_t* idx, int32_t* cnt, int kmax, int kept,
                         int nsink, const Geo& g, cudaStream_t s) {
-  if (g.Nb > kMaxNb) return cudaErrorNotSupported;
-  const long long rows = (long long)g.B * g.heads * g.Nb;
-  const long long grid = (rows + kTopkRows - 1) / kTopkRows;
-  const size_t smem = (size_t)kTopkRows * topk_stride(g.Nb) * sizeof(uint32_t);
-  static int configured_device = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_device != dev) {
-    const int max_smem = kTopkRows * topk_stride(kMaxNb) * (int)sizeof(uint32_t);
-    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
-  topk_kernel<<<(unsigned)grid, 32, smem, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
+  if (g.Nb > kMaxPerLane * 32) return cudaErrorNotSupported;
+  long long rows = (long long)g.B * g.heads * g.Nb;
+  long long grid = (rows + kTopkWarps - 1) / kTopkWarps;
+  // keys per lane: the smallest instance that covers Nb (each unused slot costs a compare
+  // and an add in every step of the search)
+  const int kpl = (g.Nb + 31) / 32;
+  const unsigned blocks = (unsigned)grid, threads = kTopkWarps * 32;
+  if (kpl <= 4)
+    topk_kernel<4><<<blocks, threads, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
+  else if (kpl <= 8)
+    topk_kernel<8><<<blocks, threads, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
+  else if (kpl <= 16)
+    topk_kernel<16><<<blocks, threads, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
+  else if (kpl <= 19)
+    topk_kernel<19><<<blocks, threads, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
+  else if (kpl <= 21)
+    topk_kernel<21><<<blocks, threads, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
+  else if (kpl <= 24)
+    topk_kernel<24><<<blocks, threads, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
+  else if (kpl <= 30)
+    topk_kernel<30><<<blocks, threads, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
+  else
+    topk_kernel<32><<<blocks, threads, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
   return cudaGetLastError();
 }
 
