@@ -115,11 +115,12 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const int4* __restri
 // ------------------------------------------------------------------------------- scores
 // One CTA per 128 x 128 tile of s for one (b, head).  D is taken 64 columns at a time:
 // the three bf16 parts of 128 query means (A) and 128 key means (B) for those columns
-// (48 KB) are loaded by TMA (128-byte swizzle, the same K-major layout as the attention
+// (96 KB) are loaded by TMA (128-byte swizzle, the same K-major layout as the attention
 // kernel's Q and K tiles) and thread 0 issues, into one fp32 TMEM accumulator, the
 // products lo.hi, hi.lo, mid.mid, mid.hi, hi.mid, hi.hi (smallest first); the dropped
-// products are below 2^-24 of the score.  With 48 KB of staging, several CTAs share an
-// SM and one's loads overlap another's products and stores.  The four warps then read
+// products are below 2^-24 of the score.  The staging is 96 KB (three parts of A and of
+// B, 16 KB each), so two CTAs share an SM and one's loads overlap the other's products
+// and stores.  The four warps then read
 // their 32 rows from TMEM and store s * scale.  Rows or columns past Nb in a tile come
 // from the next head's means (or TMA zero fill) and are not stored.
 constexpr int kSTile = 128;
