@@ -6,9 +6,10 @@
 // (batch, head, block):
 //   quant_fp8_kernel : per block, amax over its real tokens and the head's D channels,
 //                      inv = 448 / amax and scale = amax / 448 (fp32, rounded), codes =
-//                      e4m3(x * inv) (round to nearest even, saturating).  Reads the
-//                      bf16 model-order window twice (the second pass from L2) and writes
-//                      the e4m3 model-order tensor.
+//                      e4m3(x * inv) (round to nearest even, saturating).  One CTA per
+//                      (block, 128 channels of the heads*D row, tensor): the window's
+//                      rows are read from HBM once into registers, reduced across the
+//                      CTA, then converted and written as the e4m3 model-order tensor.
 //   sparse_attn_fp8_kernel : the warp-specialised pipeline of the bf16 kernel with
 //                      - S = Q K^T on e4m3 operands (kind::f8f6f4, K = 32 per MMA), the
 //                        per-block scales sq * sk_j applied to the fp32 scores;
@@ -107,20 +108,36 @@ constexpr uint32_t idesc_e4m3_f32(int M, int N, int b_mn_major) {
 }
 
 // ------------------------------------------------------------------------------ quantise
-constexpr int kQuantThreads = 128;
+constexpr int kQuantThreads = 256;
+constexpr int kQuantCols = 16;                                 // 16-byte chunks per row and CTA (128 channels)
+constexpr int kQuantItems = 128 * kQuantCols / kQuantThreads;  // chunks per thread (blk <= 128)
 
-// CTA = (128 chunks of 8 channels, block j, b * 3 + tensor).  Thread c owns channels
-// 8c .. 8c+7 of the heads*D row; the D/8 threads of a head are consecutive lanes.
+// CTA = (128 channels of the heads*D row = 128 / D heads, block j, b * 3 + tensor).  The
+// window's real rows x 16 chunks are numbered r * 16 + c and thread t owns chunks t,
+// t + 256, ...: its column c = t % 16 (so its head) is fixed, and each warp-wide copy
+// covers two whole 256-byte row slices.  Every owned chunk is copied from HBM into shared
+// memory with cp.async (no registers held while the copies are in flight, so six CTAs
+// per SM keep ~190 KB of reads outstanding), the amax of each head is reduced over the
+// lanes and then over the 8 warps, and each thread converts its own chunks from shared
+// memory and stores the codes.  Q, K and V are read once; the window's row offsets come
+// from a per-CTA table.
 template <int D>
 __global__ void __launch_bounds__(kQuantThreads) quant_fp8_kernel(const int4* __restrict__ q, const int4* __restrict__ k,
                                                                  const int4* __restrict__ v, uint8_t* __restrict__ q8,
                                                                  uint8_t* __restrict__ k8, uint8_t* __restrict__ v8,
                                                                  float* __restrict__ scales, Geo g, int chunks) {
-  constexpr int kPerHead = D / 8;
-  const int c = blockIdx.x * kQuantThreads + threadIdx.x;
+  constexpr int kPerHead = D / 8;                // chunks of one head's row
+  constexpr int kHeads = kQuantCols / kPerHead;  // heads per CTA
+  __shared__ __align__(16) int4 stage[kQuantItems * kQuantThreads];
+  __shared__ int roff_s[128];
+  __shared__ float red[kQuantThreads / 32][kHeads];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = tid & (kQuantCols - 1);
+  const int hl = c / kPerHead;  // head within the CTA
+  const int head0 = blockIdx.x * kHeads;
+  const bool col_live = head0 + hl < g.heads;
   const int j = blockIdx.y;
   const int b = blockIdx.z / 3, t = blockIdx.z - b * 3;
-  const bool live = c < chunks;
   const int4* src = (t == 0 ? q : t == 1 ? k : v);
   uint8_t* dst = (t == 0 ? q8 : t == 1 ? k8 : v8);
   int nt, nh, nw;
@@ -129,46 +146,74 @@ __global__ void __launch_bounds__(kQuantThreads) quant_fp8_kernel(const int4* __
   const int tb = j / per_t, hb = (j - tb * per_t) / g.nbw, wb = j - tb * per_t - hb * g.nbw;
   const long long row0 = (long long)b * g.N + ((long long)tb * g.wt * g.H + (long long)hb * g.wh) * g.W +
                          (long long)wb * g.ww;
-  const long long t_stride = (long long)g.H * g.W, h_stride = g.W;
-  float amax = 0.f;
-  if (live) {
-    for (int dt = 0; dt < nt; ++dt)
-      for (int dh = 0; dh < nh; ++dh) {
-        const long long r0 = row0 + dt * t_stride + dh * h_stride;
-        for (int dw = 0; dw < nw; ++dw) {
-          const int4 x = __ldg(src + (r0 + dw) * chunks + c);
-          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&x);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(h2[e]);
-            amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
-          }
-        }
-      }
+  const int rows = nt * nh * nw;
+  // token offset of each real row of the window from its first token (-1 past the real
+  // rows), computed once per CTA: dividing per chunk costs more issue slots than the copy
+  if (tid < 128) {
+    int o = -1;
+    if (tid < rows) {
+      const int dw = tid % nw, rest = tid / nw;
+      const int dh = rest % nh, dt = rest / nh;
+      o = (int)(dt * (long long)g.H * g.W + dh * (long long)g.W + dw);
+    }
+    roff_s[tid] = o;
   }
+  __syncthreads();
+  // chunk index of the window's first token at this thread's column; a chunk is addressed
+  // by its token offset from there (< B * N < 2^31)
+  const long long base = row0 * chunks + (long long)head0 * kPerHead + c;
+  const int rsub = tid / kQuantCols;
 #pragma unroll
-  for (int o = 1; o < kPerHead; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  if (!live) return;
-  const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
-  const int head = c / kPerHead;
-  if (c % kPerHead == 0)
-    scales[(((long long)t * g.B + b) * g.heads + head) * g.Nb + j] = amax > 0.f ? __fdiv_rn(amax, 448.f) : 0.f;
-  for (int dt = 0; dt < nt; ++dt)
-    for (int dh = 0; dh < nh; ++dh) {
-      const long long r0 = row0 + dt * t_stride + dh * h_stride;
-      for (int dw = 0; dw < nw; ++dw) {
-        const int4 x = __ldg(src + (r0 + dw) * chunks + c);
-        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&x);
-        uint32_t w[2];
+  for (int it = 0; it < kQuantItems; ++it) {
+    const int ro = roff_s[rsub + it * (kQuantThreads / kQuantCols)];
+    if (ro >= 0 && col_live) {
+      const uint32_t sdst = ptx::smem_u32(&stage[it * kQuantThreads + tid]);
+      const int4* gsrc = src + base + (long long)ro * chunks;
+      asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16;" ::"r"(sdst), "l"(gsrc) : "memory");
+    }
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  float amax = 0.f;
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float2 f0 = __bfloat1622float2(h2[2 * e]), f1 = __bfloat1622float2(h2[2 * e + 1]);
-          w[e] = e4m3x2(__fmul_rn(f0.x, inv), __fmul_rn(f0.y, inv)) |
-                 (e4m3x2(__fmul_rn(f1.x, inv), __fmul_rn(f1.y, inv)) << 16);
-        }
-        *reinterpret_cast<uint2*>(dst + ((r0 + dw) * chunks + c) * 8) = make_uint2(w[0], w[1]);
+  for (int it = 0; it < kQuantItems; ++it) {
+    if (roff_s[rsub + it * (kQuantThreads / kQuantCols)] >= 0 && col_live) {
+      const int4 x = stage[it * kQuantThreads + tid];
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&x);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h2[e]);
+        amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
       }
     }
+  }
+  // lanes l and l ^ 16 hold the same column; the kPerHead columns of a head are adjacent
+#pragma unroll
+  for (int o = 1; o < kPerHead; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
+  if (lane < kQuantCols && (lane % kPerHead) == 0) red[warp][hl] = amax;
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < kQuantThreads / 32; ++w) amax = fmaxf(amax, red[w][hl]);
+  if (!col_live) return;
+  const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
+  if (tid < kQuantCols && c % kPerHead == 0)
+    scales[(((long long)t * g.B + b) * g.heads + head0 + hl) * g.Nb + j] = amax > 0.f ? __fdiv_rn(amax, 448.f) : 0.f;
+#pragma unroll
+  for (int it = 0; it < kQuantItems; ++it) {
+    const int ro = roff_s[rsub + it * (kQuantThreads / kQuantCols)];
+    if (ro >= 0) {
+      const int4 x = stage[it * kQuantThreads + tid];
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&x);
+      uint32_t w[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float2 f0 = __bfloat1622float2(h2[2 * e]), f1 = __bfloat1622float2(h2[2 * e + 1]);
+        w[e] = e4m3x2(__fmul_rn(f0.x, inv), __fmul_rn(f0.y, inv)) |
+               (e4m3x2(__fmul_rn(f1.x, inv), __fmul_rn(f1.y, inv)) << 16);
+      }
+      *reinterpret_cast<uint2*>(dst + (base + (long long)ro * chunks) * 8) = make_uint2(w[0], w[1]);
+    }
+  }
 }
 
 // ------------------------------------------------------------------------------ attention
@@ -640,7 +685,8 @@ cudaError_t launch_quant_fp8(const void* q, const void* k, const void* v, uint8_
                              float* scales, const Geo& g, cudaStream_t s) {
   if (g.D != 128 && g.D != 64) return cudaErrorNotSupported;
   const int chunks = g.heads * g.D / 8;
-  dim3 grid((chunks + kQuantThreads - 1) / kQuantThreads, g.Nb, g.B * 3);
+  const int heads_per_cta = kQuantCols / (g.D / 8);
+  dim3 grid((g.heads + heads_per_cta - 1) / heads_per_cta, g.Nb, g.B * 3);
   if (g.D == 128)
     quant_fp8_kernel<128><<<grid, kQuantThreads, 0, s>>>((const int4*)q, (const int4*)k, (const int4*)v, q8, k8, v8,
                                                           scales, g, chunks);

@@ -120,9 +120,10 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const int4* __restri
 // products lo.hi, hi.lo, mid.mid, mid.hi, hi.mid, hi.hi (smallest first); the dropped
 // products are below 2^-24 of the score.  The staging is 96 KB (three parts of A and of
 // B, 16 KB each), so two CTAs share an SM and one's loads overlap the other's products
-// and stores.  The four warps then read
-// their 32 rows from TMEM and store s * scale.  Rows or columns past Nb in a tile come
-// from the next head's means (or TMA zero fill) and are not stored.
+// and stores.  The four warps then read their 32 rows from TMEM and store s * scale,
+// turned around in the freed staging so that stores cover whole 128-byte row segments
+// (when Nb is a multiple of 4; else element by element).  Rows or columns past Nb in a
+// tile come from the next head's means (or TMA zero fill) and are not stored.
 constexpr int kSTile = 128;
 constexpr int kSThreads = 128;
 constexpr uint64_t kScoresWaitNs = 500ull * 1000ull * 1000ull;
@@ -169,6 +170,8 @@ __global__ void __launch_bounds__(kSThreads) scores_kernel(const __grid_constant
   ptx::tc_fence_after();
   const uint32_t tmem = tmem_slot;
   volatile int* abort_flag = &abort_s;
+  // the block means come from the pool kernel, which may still be finishing
+  ptx::grid_dep_wait();
   if (threadIdx.x == 0) {
     ptx::prefetch_tmap(&ta);
     ptx::prefetch_tmap(&tb);
@@ -219,21 +222,40 @@ __global__ void __launch_bounds__(kSThreads) scores_kernel(const __grid_constant
     ptx::tc_fence_after();
     const int r = warp * 32 + lane;  // tile row == TMEM lane
     const int gi = i0 + r;
-    float* srow = s + (bh * g.Nb + gi) * (long long)g.Nb + j0;
-    const bool vec = (g.Nb & 3) == 0;
+    if ((g.Nb & 3) == 0) {
+      // Every MMA has completed, so the operand staging is free: each warp turns its 32 x 32
+      // chunk around in shared memory (rows padded to 33 words: no bank conflicts either
+      // way) and eight lanes then store one whole 128-byte row segment, so no L2 sector is
+      // left half written.
+      float* tr = reinterpret_cast<float*>(smem) + warp * (32 * 33);
+      const int rr0 = lane >> 3, cc = 4 * (lane & 7);
 #pragma unroll 1
-    for (int c = 0; c < kSTile / 32; ++c) {
-      uint32_t v[32];
-      ptx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c * 32, v);
-      if (gi < g.Nb) {
-        const int cb = c * 32;
-        if (vec && j0 + cb + 32 <= g.Nb) {
+      for (int c = 0; c < kSTile / 32; ++c) {
+        uint32_t v[32];
+        ptx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c * 32, v);
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            reinterpret_cast<float4*>(srow + cb)[e] =
-                make_float4(__uint_as_float(v[4 * e]) * scale, __uint_as_float(v[4 * e + 1]) * scale,
-                            __uint_as_float(v[4 * e + 2]) * scale, __uint_as_float(v[4 * e + 3]) * scale);
-        } else {
+        for (int e = 0; e < 32; ++e) tr[lane * 33 + e] = __uint_as_float(v[e]) * scale;
+        __syncwarp();
+        const int gj = j0 + c * 32 + cc;  // gj % 4 == 0 and Nb % 4 == 0: gj < Nb covers gj + 3
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 4 * i + rr0;
+          const int gr = i0 + warp * 32 + rr;
+          if (gr < g.Nb && gj < g.Nb) {
+            const float* t = tr + rr * 33 + cc;
+            *reinterpret_cast<float4*>(s + (bh * g.Nb + gr) * (long long)g.Nb + gj) = make_float4(t[0], t[1], t[2], t[3]);
+          }
+        }
+        __syncwarp();
+      }
+    } else {
+      float* srow = s + (bh * g.Nb + gi) * (long long)g.Nb + j0;
+#pragma unroll 1
+      for (int c = 0; c < kSTile / 32; ++c) {
+        uint32_t v[32];
+        ptx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c * 32, v);
+        if (gi < g.Nb) {
+          const int cb = c * 32;
 #pragma unroll
           for (int e = 0; e < 32; ++e)
             if (j0 + cb + e < g.Nb) srow[cb + e] = __uint_as_float(v[e]) * scale;
@@ -272,10 +294,93 @@ __device__ __forceinline__ int count_ge(const uint32_t (&key)[KPL], uint32_t t) 
   return (int)__reduce_add_sync(0xffffffffu, (uint32_t)c);
 }
 
+// Score of an order key (the inverse of order_key).
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Histogram bin of a key: fma(v, sc, off) clamped to [0, 63] and rounded to an integer by
+// adding 1.5 * 2^23 (the sum's low mantissa bits are the rounded value).  Each step is
+// monotone in v, so the bin never decreases as the key grows; equal keys share a bin.
+__device__ __forceinline__ int bin_index(uint32_t k, float sc, float off) {
+  const float x = fminf(fmaxf(__fmaf_rn(key_value(k), sc, off), 0.f), 63.f);
+  return __float_as_int(__fadd_rn(x, 12582912.f)) & 63;
+}
+
+// Cut of a row from a 64-bin histogram of the candidate scores, linear in value between
+// the row's smallest and largest score.  The bin of a key, min(63, max(0, trunc(fma(v,
+// sc, off)))), never decreases as the key grows and equal keys share a bin, so the m-th
+// largest key lies in the bin where the count of keys in it and above first reaches m;
+// that bin's keys (at most 32, else this returns false and the caller searches) are
+// gathered one per lane and ranked exactly.  On success thr is the m-th largest key,
+// above = #{key > thr} and eqc = #{key == thr}.
+template <int KPL>
+__device__ __forceinline__ bool cut_by_histogram(const uint32_t (&key)[KPL], uint32_t lo_key, uint32_t hi_key,
+                                                 int m, uint32_t* hist, uint32_t* list, int lane, uint32_t& thr,
+                                                 int& above, int& eqc) {
+  const float vmin = key_value(lo_key), vmax = key_value(hi_key);
+  const float sc = 64.f / (vmax - vmin);
+  const float off = -vmin * sc;
+  // equal ends (one bin), or ends whose range does not give finite bin arithmetic
+  if (!(vmax > vmin) || !(sc <= 3.0e38f) || !(fabsf(off) <= 3.0e38f)) return false;
+  reinterpret_cast<uint2*>(hist)[lane] = make_uint2(0u, 0u);
+  __syncwarp();
+  int bin[KPL];
+#pragma unroll
+  for (int k = 0; k < KPL; ++k) {
+    bin[k] = bin_index(key[k], sc, off);
+    if (key[k] != 0u) atomicAdd(&hist[bin[k]], 1u);
+  }
+  __syncwarp();
+  const uint2 cc = reinterpret_cast<const uint2*>(hist)[lane];  // bins 2 lane, 2 lane + 1
+  uint32_t suf = cc.x + cc.y;                                    // keys in bins >= 2 lane
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_down_sync(0xffffffffu, suf, o);
+    if (lane + o < 32) suf += t;
+  }
+  const uint32_t suf_hi = suf - cc.x;                            // keys in bins >= 2 lane + 1
+  // suf never grows with the lane; lane 0 holds every candidate (> m)
+  const int L = 31 - __clz(__ballot_sync(0xffffffffu, suf >= (uint32_t)m));
+  const bool upper = suf_hi >= (uint32_t)m;
+  const int B_l = 2 * lane + (upper ? 1 : 0);
+  const int nB_l = (int)(upper ? cc.y : cc.x);
+  const int ab_l = (int)(upper ? suf_hi - cc.y : suf_hi);        // keys in bins above B
+  const int B = __shfl_sync(0xffffffffu, B_l, L);
+  const int nB = __shfl_sync(0xffffffffu, nB_l, L);
+  const int ab = __shfl_sync(0xffffffffu, ab_l, L);
+  if (nB > 32) return false;
+  const int r = m - ab;  // rank of the cut inside bin B, 1 <= r <= nB
+  int cnt = 0;
+#pragma unroll
+  for (int k = 0; k < KPL; ++k) {
+    const bool in = key[k] != 0u && bin[k] == B;
+    const uint32_t bal = __ballot_sync(0xffffffffu, in);
+    if (in) list[cnt + __popc(bal & ((1u << lane) - 1u))] = key[k];
+    cnt += __popc(bal);
+  }
+  __syncwarp();
+  const uint32_t x = lane < nB ? list[lane] : 0u;
+  int gt = 0, ge = 0;
+#pragma unroll 1
+  for (int i = 0; i < nB; ++i) {
+    const uint32_t y = __shfl_sync(0xffffffffu, x, i);
+    gt += y > x;
+    ge += y >= x;
+  }
+  const uint32_t hit = __ballot_sync(0xffffffffu, lane < nB && gt < r && ge >= r);
+  const int src = __ffs(hit) - 1;
+  thr = __shfl_sync(0xffffffffu, x, src);
+  const int g = __shfl_sync(0xffffffffu, gt, src), e = __shfl_sync(0xffffffffu, ge, src);
+  above = ab + g;
+  eqc = e - g;
+  return true;
+}
+
 template <int KPL>
 __device__ __forceinline__ void topk_row(const float* __restrict__ sr, int32_t* __restrict__ out,
                                          int32_t* __restrict__ cnt_out, int Nb, int kmax, int kept,
-                                         int nsink, int lane) {
+                                         int nsink, int lane, uint32_t* hist, uint32_t* list) {
   uint32_t key[KPL];
   uint32_t kmin = 0xffffffffu, kmax_key = 0u;
 #pragma unroll
@@ -288,95 +393,87 @@ __device__ __forceinline__ void topk_row(const float* __restrict__ sr, int32_t* 
   const int m = kept - nsink;
   const int ncand = Nb - nsink;
   uint32_t thr;       // every candidate key >= thr is kept when take_eq covers all keys == thr
+  int above = 0, eqc = 0;
   if (m <= 0) {
     thr = 0xffffffffu;  // none (no real key reaches the top value: keys are < 2^32 - 1 or
                         // equal to it only for NaN patterns, which the ordering puts last)
   } else if (m >= ncand) {
     thr = 1u;           // every candidate
   } else {
-    // Bracket [lo, hi): #{key >= lo} = c_lo >= m > c_hi = #{key >= hi}.  Each step tries a
-    // t inside the bracket, interpolated from the two counts (keys of a smooth score
-    // distribution are close to uniform locally) on even steps and the midpoint on odd
-    // steps, and stops when exactly m keys are >= t.  Otherwise the bracket shrinks to
-    // one value: lo is then the m-th largest key.
-    uint64_t lo = __reduce_min_sync(0xffffffffu, kmin);
-    uint64_t hi = (uint64_t)__reduce_max_sync(0xffffffffu, kmax_key) + 1u;
-    int c_lo = ncand, c_hi = 0;
-    bool exact = false;
+    const uint32_t lo_key = __reduce_min_sync(0xffffffffu, kmin);
+    const uint32_t hi_key = __reduce_max_sync(0xffffffffu, kmax_key);
+    if (!cut_by_histogram<KPL>(key, lo_key, hi_key, m, hist, list, lane, thr, above, eqc)) {
+      // Bracket [lo, hi): #{key >= lo} = c_lo >= m > c_hi = #{key >= hi}.  Each step tries
+      // a t inside the bracket, interpolated from the two counts on even steps and the
+      // midpoint on odd steps, and stops when exactly m keys are >= t.  Otherwise the
+      // bracket shrinks to one value: lo is then the m-th largest key.
+      uint64_t lo = lo_key;
+      uint64_t hi = (uint64_t)hi_key + 1u;
+      int c_lo = ncand, c_hi = 0;
 #pragma unroll 1
-    for (int step = 0; hi - lo > 1; ++step) {
-      const uint64_t w = hi - lo;
-      uint64_t off;
-      if (step & 1) {
-        off = w >> 1;
-      } else {
-        const float frac = (float)(c_lo - m) / (float)(c_lo - c_hi);
-        off = (uint64_t)((double)w * (double)frac);
+      for (int step = 0; hi - lo > 1; ++step) {
+        const uint64_t w = hi - lo;
+        uint64_t off;
+        if (step & 1) {
+          off = w >> 1;
+        } else {
+          const float frac = (float)(c_lo - m) / (float)(c_lo - c_hi);
+          off = (uint64_t)((double)w * (double)frac);
+        }
+        off = off < 1 ? 1 : (off > w - 1 ? w - 1 : off);
+        const uint32_t t = (uint32_t)(lo + off);
+        const int c = count_ge<KPL>(key, t);
+        if (c == m) {
+          lo = t;
+          break;
+        }
+        if (c > m) {
+          lo = t;
+          c_lo = c;
+        } else {
+          hi = t;
+          c_hi = c;
+        }
       }
-      off = off < 1 ? 1 : (off > w - 1 ? w - 1 : off);
-      const uint32_t t = (uint32_t)(lo + off);
-      const int c = count_ge<KPL>(key, t);
-      if (c == m) {
-        lo = t;
-        exact = true;
-        break;
-      }
-      if (c > m) {
-        lo = t;
-        c_lo = c;
-      } else {
-        hi = t;
-        c_hi = c;
-      }
-    }
-    (void)exact;
-    thr = (uint32_t)lo;
-  }
-  // keys above thr are kept; of the keys equal to thr, the take_eq lowest ids
-  int above = 0, eqc = 0;
+      thr = (uint32_t)lo;
 #pragma unroll
-  for (int k = 0; k < KPL; ++k) {
-    above += key[k] > thr;
-    eqc += key[k] == thr;
+      for (int k = 0; k < KPL; ++k) {
+        above += key[k] > thr;
+        eqc += key[k] == thr;
+      }
+      above = (int)__reduce_add_sync(0xffffffffu, (uint32_t)above);
+      eqc = (int)__reduce_add_sync(0xffffffffu, (uint32_t)eqc);
+    }
   }
-  above = (int)__reduce_add_sync(0xffffffffu, (uint32_t)above);
-  eqc = (int)__reduce_add_sync(0xffffffffu, (uint32_t)eqc);
-  const bool all = m >= ncand;
-  const bool some = m > 0 && m < ncand;
-  const int take_eq = some ? m - above : 0;
-  int pos = 0;
-  if (!some || take_eq == eqc) {
-    // every key equal to thr is kept (or none is): one ballot per 32 blocks
+  // The sink blocks are ids 0 .. nsink - 1, the smallest, so the list starts with them.
+  // Candidates (key != 0) above thr are kept; of those equal to thr, the take_eq lowest
+  // ids (all of them when take_eq == eqc).  thr = 1 keeps every candidate.
+  const int ns = min(nsink, kmax);
+  for (int p = lane; p < ns; p += 32) out[p] = p;
+  int pos = nsink;
+  const int take_eq = (m > 0 && m < ncand) ? m - above : 0;
+  if (m > 0 && (m >= ncand || take_eq == eqc)) {
 #pragma unroll
     for (int k = 0; k < KPL; ++k) {
       if (k * 32 >= Nb) break;
-      const int j = k * 32 + lane;
-      const bool in_range = j < Nb;
-      const bool is_sink = in_range && j < nsink;
-      const bool cand = in_range && !is_sink && key[k] != 0u;
-      const bool take = is_sink || (cand && (all || (some && key[k] >= thr)));
+      const bool take = key[k] >= thr;  // pad and sink slots hold key 0 < thr
       const uint32_t tmask = __ballot_sync(0xffffffffu, take);
       const int p = pos + __popc(tmask & ((1u << lane) - 1u));
-      if (take && p < kmax) out[p] = j;
+      if (take && p < kmax) out[p] = k * 32 + lane;
       pos += __popc(tmask);
     }
-  } else {
+  } else if (m > 0) {
     int eq_taken = 0;
 #pragma unroll
     for (int k = 0; k < KPL; ++k) {
       if (k * 32 >= Nb) break;
-      const int j = k * 32 + lane;
-      const bool in_range = j < Nb;
-      const bool is_sink = in_range && j < nsink;
-      const bool gt = in_range && !is_sink && key[k] > thr;
-      const bool eq = in_range && !is_sink && key[k] == thr;
+      const bool eq = key[k] == thr;
       const uint32_t eqmask = __ballot_sync(0xffffffffu, eq);
-      const int eq_rank = eq_taken + __popc(eqmask & ((1u << lane) - 1u));
-      const bool take = is_sink || gt || (eq && eq_rank < take_eq);
+      const bool take = key[k] > thr || (eq && eq_taken + __popc(eqmask & ((1u << lane) - 1u)) < take_eq);
       eq_taken += __popc(eqmask);
       const uint32_t tmask = __ballot_sync(0xffffffffu, take);
       const int p = pos + __popc(tmask & ((1u << lane) - 1u));
-      if (take && p < kmax) out[p] = j;
+      if (take && p < kmax) out[p] = k * 32 + lane;
       pos += __popc(tmask);
     }
   }
@@ -390,11 +487,32 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
                                                                int32_t* __restrict__ cnt,
                                                                int Nb, long long rows, int kmax,
                                                                int kept, int nsink) {
+  __shared__ __align__(8) uint32_t hist_s[kTopkWarps][64];
+  __shared__ uint32_t list_s[kTopkWarps][32];
   const int lane = threadIdx.x & 31;
   const int w = threadIdx.x >> 5;
   const long long row = (long long)blockIdx.x * kTopkWarps + w;
+  ptx::grid_dep_wait();  // the scores come from the scores kernel, which may still be finishing
   if (row >= rows) return;
-  topk_row<KPL>(s + row * Nb, idx + row * kmax, cnt + row, Nb, kmax, kept, nsink, lane);
+  topk_row<KPL>(s + row * Nb, idx + row * kmax, cnt + row, Nb, kmax, kept, nsink, lane, hist_s[w], list_s[w]);
+}
+
+// Launch with programmatic stream serialization (the kernel waits for its predecessor
+// in the stream with grid_dep_wait before it reads that kernel's output).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
 }  // namespace
@@ -439,8 +557,7 @@ cudaError_t launch_scores_d(const __nv_bfloat16* q3, const __nv_bfloat16* k3, fl
     configured_device = dev;
   }
   dim3 grid((g.Nb + kSTile - 1) / kSTile, (g.Nb + kSTile - 1) / kSTile, g.B * g.heads);
-  scores_kernel<D><<<grid, kSThreads, C::kSmem, s>>>(ta, tb, scores, g, scale, status);
-  return cudaGetLastError();
+  return launch_dependent(scores_kernel<D>, grid, dim3(kSThreads), C::kSmem, s, ta, tb, scores, g, scale, status);
 }
 
 cudaError_t launch_scores(const __nv_bfloat16* q3, const __nv_bfloat16* k3, float* scores, const Geo& g,
@@ -454,27 +571,28 @@ cudaError_t launch_topk(const float* scores, int32_t* idx, int32_t* cnt, int kma
   if (g.Nb > kMaxPerLane * 32) return cudaErrorNotSupported;
   long long rows = (long long)g.B * g.heads * g.Nb;
   long long grid = (rows + kTopkWarps - 1) / kTopkWarps;
-  // keys per lane: the smallest instance that covers Nb (each unused slot costs a compare
-  // and an add in every step of the search)
+  // keys per lane: the smallest instance that covers Nb (each unused slot costs
+  // instructions in every pass over the keys)
   const int kpl = (g.Nb + 31) / 32;
   const unsigned blocks = (unsigned)grid, threads = kTopkWarps * 32;
+  cudaError_t e;
   if (kpl <= 4)
-    topk_kernel<4><<<blocks, threads, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
+    e = launch_dependent(topk_kernel<4>, dim3(blocks), dim3(threads), 0, s, scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
   else if (kpl <= 8)
-    topk_kernel<8><<<blocks, threads, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
+    e = launch_dependent(topk_kernel<8>, dim3(blocks), dim3(threads), 0, s, scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
   else if (kpl <= 16)
-    topk_kernel<16><<<blocks, threads, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
+    e = launch_dependent(topk_kernel<16>, dim3(blocks), dim3(threads), 0, s, scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
   else if (kpl <= 19)
-    topk_kernel<19><<<blocks, threads, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
+    e = launch_dependent(topk_kernel<19>, dim3(blocks), dim3(threads), 0, s, scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
   else if (kpl <= 21)
-    topk_kernel<21><<<blocks, threads, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
+    e = launch_dependent(topk_kernel<21>, dim3(blocks), dim3(threads), 0, s, scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
   else if (kpl <= 24)
-    topk_kernel<24><<<blocks, threads, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
+    e = launch_dependent(topk_kernel<24>, dim3(blocks), dim3(threads), 0, s, scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
   else if (kpl <= 30)
-    topk_kernel<30><<<blocks, threads, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
+    e = launch_dependent(topk_kernel<30>, dim3(blocks), dim3(threads), 0, s, scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
   else
-    topk_kernel<32><<<blocks, threads, 0, s>>>(scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
-  return cudaGetLastError();
+    e = launch_dependent(topk_kernel<32>, dim3(blocks), dim3(threads), 0, s, scores, idx, cnt, g.Nb, rows, kmax, kept, nsink);
+  return e;
 }
 
 }  // namespace rf2

@@ -76,6 +76,55 @@ def test_predict_mask_exact_ties_take_the_lowest_ids(shape, raster):
         assert np.array_equal(got.reshape(-1, sel.kept), np.broadcast_to(np.arange(sel.kept), (got.size // sel.kept, sel.kept)))
 
 
+# 192 blocks of 64 tokens, 48 of them the first-frame sink: 144 candidates per row, enough
+# for the cut's histogram bin to overflow its 32 slots when the scores crowd together.
+CUT_SHAPE = dict(B=1, heads=2, T=4, H=48, W=64, D=64, wt=1, wh=8, ww=8)
+
+
+def _block_ids(og):
+    """Window block of every model-order token, [N]."""
+    t, h, w = np.meshgrid(np.arange(og.T), np.arange(og.H), np.arange(og.W), indexing="ij")
+    nbh, nbw = -(-og.H // og.wh), -(-og.W // og.ww)
+    return (((t // og.wt) * nbh + h // og.wh) * nbw + w // og.ww).reshape(-1)
+
+
+@pytest.mark.parametrize("case", ["outlier_column", "levels3", "levels9"])
+def test_predict_mask_cut_by_histogram_and_by_search(case):
+    """Rows whose cut the top-k finds through its value histogram and rows where it must
+    fall back to the bracketed search give the oracle's lists.  outlier_column: one key
+    block scaled by 512 takes one end of every row's score range, so the other 143 scores
+    share one or two of the 64 bins and the cut's bin overflows (search); the lists are
+    compared outside the near-cut window.  levelsL: every key block mean is c u for one
+    vector u and an integer c in [-(L-1)/2, (L-1)/2], so each row has L distinct scores,
+    exact ties in fp64 and in the kernel's fp32, and the lists must equal the oracle's
+    (lowest ids among equal scores) bit for bit: with 3 levels about 48 candidates share
+    the cut's score (search), with 9 about 16 (histogram)."""
+    from rf2_inputs import f32_to_bf16_bits
+    g, og = rf2.Geometry(**CUT_SHAPE), O.geom(**CUT_SHAPE)
+    q, k, _ = _rand_bits(g, 1600)
+    rng = np.random.default_rng(1601)
+    blocks = _block_ids(og)
+    if case == "outlier_column":
+        kf = bf16_bits_to_f64(k).astype(np.float32)
+        kf[:, blocks == 100] *= 512.0   # a non-sink block; a power of two keeps bf16 exact
+    else:
+        u = rng.standard_normal((g.heads, g.D)).astype(np.float32)
+        half = (int(case[len("levels"):]) - 1) // 2
+        level = rng.integers(-half, half + 1, size=int(blocks.max()) + 1).astype(np.float32)
+        kf = (level[blocks][None, :, None, None] * u[None, None]).astype(np.float32)
+        kf = np.broadcast_to(kf, (g.B, g.N, g.heads, g.D))
+    k = f32_to_bf16_bits(np.ascontiguousarray(kf))
+    qp, kp = O.permute(q, og), O.permute(k, og)
+    for s_, sink in ((0.8, True), (0.6, False), (0.9, True)):
+        sel = O.predict_mask(bf16_bits_to_f64(qp), bf16_bits_to_f64(kp), og, s_, sink)
+        idx, cnt = rf2.predict_mask(to_dev(q), to_dev(k), g, s_, sink, checked=True, raster=True)
+        if case == "outlier_column":
+            compare_lists(idx.cpu().numpy(), cnt.cpu().numpy(), sel)
+        else:
+            assert np.array_equal(idx.cpu().numpy(), sel.idx), (s_, sink)
+            assert np.all(cnt.cpu().numpy() == sel.kept)
+
+
 @pytest.mark.parametrize("shape", RAGGED)
 def test_permute_unpermute_ragged_bit_exact(shape):
     g, og = rf2.Geometry(**shape), O.geom(**shape)
