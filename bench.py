@@ -552,6 +552,28 @@ def main():
     del xp
     peaks = _peaks()
 
+    # The mask stage alone: rf2_predict_mask back to back (its inputs as in the step).  In
+    # the step it follows the previous attention call, whose output is still dirty in L2
+    # and whose clock is the power-capped one; this isolates the mask kernels' own rate.
+    best = float("nan")
+    try:
+        times = []
+        for rep in range(4):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            ev[0].record(stream)
+            for _ in range(10):
+                rf2.predict_mask(q, k, g, sparsity, wl.sink, kmax=kept, ws=mws, out=(idx, cnt), raster=True)
+            ev[1].record(stream)
+            torch.cuda.synchronize(dev)
+            if rep:  # the first repetition warms up
+                times.append(ev[0].elapsed_time(ev[1]) / 10)
+        best = min(times)
+    except Exception as exc:  # a measurement for the record only: never fail the bench on it
+        print(f"mask stage alone not measured: {exc}", file=sys.stderr)
+    mask_alone_ms = max_over_ranks([best], dev)[0]  # every rank takes part, measured or not
+    if not math.isfinite(mask_alone_ms):
+        mask_alone_ms = None
+
     # end to end through the public fused call: pinned host inputs in, host output back
     e2e = None
     if not a.no_e2e:
@@ -645,6 +667,10 @@ def main():
         "stages_ms": {"predict_mask": seg_ms[0], "sparse_attn": seg_ms[1]},
         "mask_stage": {"ms": seg_ms[0], "GB/s": mask_gbs, "frac_hbm": mask_gbs / peaks["hbm_gbs"],
                        "bytes": mask_bytes},
+        "mask_stage_alone": (None if mask_alone_ms is None else
+                             {"ms": mask_alone_ms, "GB/s": mask_bytes / (mask_alone_ms * 1e-3) / 1e9,
+                              "frac_hbm": mask_bytes / (mask_alone_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                              "note": "rf2_predict_mask back to back, best of 3 x 10 calls"}),
         "permute_kernels": {"note": "stand-alone rf2_permute x3 / rf2_unpermute, outside the step",
                             "permute_qkv_ms": perm_ms, "permute_GB/s": perm_bytes / (perm_ms * 1e-3) / 1e9,
                             "unpermute_ms": unperm_ms,

@@ -16,6 +16,12 @@
 namespace rf2 {
 namespace {
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization
+// may start while the kernel before it in the stream is finishing; grid_dep_wait blocks
+// (in hardware) until that kernel has completed and its writes are visible.  It is a no-op
+// for a kernel launched without the attribute.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------------------- pool
 // CTA = (16-byte chunk group of 128 chunks = 1024 channels, block j, b*2 + tensor).
 // Each thread owns one 16-byte chunk (8 channels) of the heads*D row and sums it over
@@ -113,7 +119,8 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const int4* __restri
 }
 
 // ------------------------------------------------------------------------------- scores
-// One CTA per 128 x 128 tile of s for one (b, head).  D is taken 64 columns at a time:
+// One CTA per 128 x 128 tile of s for one (b, head); the column tiles start at the sink
+// boundary rounded down to 32 (the top-k reads no sink column).  D is taken 64 columns at a time:
 // the three bf16 parts of 128 query means (A) and 128 key means (B) for those columns
 // (96 KB) are loaded by TMA (128-byte swizzle, the same K-major layout as the attention
 // kernel's Q and K tiles) and thread 0 issues, into one fp32 TMEM accumulator, the
@@ -125,7 +132,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const int4* __restri
 // (when Nb is a multiple of 4; else element by element).  Rows or columns past Nb in a
 // tile come from the next head's means (or TMA zero fill) and are not stored.
 constexpr int kSTile = 128;
-constexpr int kSThreads = 128;
+constexpr int kSThreads = 256;
 constexpr uint64_t kScoresWaitNs = 500ull * 1000ull * 1000ull;
 
 template <int D>
@@ -142,7 +149,7 @@ template <int D>
 __global__ void __launch_bounds__(kSThreads) scores_kernel(const __grid_constant__ CUtensorMap ta,
                                                               const __grid_constant__ CUtensorMap tb,
                                                               float* __restrict__ s, Geo g, float scale,
-                                                              int* __restrict__ status) {
+                                                              int jbase, int* __restrict__ status) {
   using C = ScoresCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -152,7 +159,7 @@ __global__ void __launch_bounds__(kSThreads) scores_kernel(const __grid_constant
   const uint32_t bar_full = sbase + C::kOffBar, bar_free = bar_full + 8, bar_done = bar_full + 16;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long bh = blockIdx.z;
-  const int i0 = blockIdx.y * kSTile, j0 = blockIdx.x * kSTile;
+  const int i0 = blockIdx.y * kSTile, j0 = jbase + blockIdx.x * kSTile;
   const long long R = (long long)g.B * g.heads * g.Nb;  // rows of one part
   if (warp == 0) {
     ptx::tmem_alloc(ptx::smem_u32(&tmem_slot), kSTile);
@@ -171,7 +178,7 @@ __global__ void __launch_bounds__(kSThreads) scores_kernel(const __grid_constant
   const uint32_t tmem = tmem_slot;
   volatile int* abort_flag = &abort_s;
   // the block means come from the pool kernel, which may still be finishing
-  ptx::grid_dep_wait();
+  grid_dep_wait();
   if (threadIdx.x == 0) {
     ptx::prefetch_tmap(&ta);
     ptx::prefetch_tmap(&tb);
@@ -220,7 +227,10 @@ __global__ void __launch_bounds__(kSThreads) scores_kernel(const __grid_constant
                   *abort_flag == 0;
   if (ok) {
     ptx::tc_fence_after();
-    const int r = warp * 32 + lane;  // tile row == TMEM lane
+    // warps w and w + 4 read TMEM lanes 32 (w % 4) .. + 31 (tile rows), each half of the
+    // columns
+    const int quad = warp & 3, c0 = (warp >> 2) * (kSTile / 64);
+    const int r = quad * 32 + lane;  // tile row == TMEM lane
     const int gi = i0 + r;
     if ((g.Nb & 3) == 0) {
       // Every MMA has completed, so the operand staging is free: each warp turns its 32 x 32
@@ -230,9 +240,9 @@ __global__ void __launch_bounds__(kSThreads) scores_kernel(const __grid_constant
       float* tr = reinterpret_cast<float*>(smem) + warp * (32 * 33);
       const int rr0 = lane >> 3, cc = 4 * (lane & 7);
 #pragma unroll 1
-      for (int c = 0; c < kSTile / 32; ++c) {
+      for (int c = c0; c < c0 + kSTile / 64; ++c) {
         uint32_t v[32];
-        ptx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c * 32, v);
+        ptx::tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + c * 32, v);
 #pragma unroll
         for (int e = 0; e < 32; ++e) tr[lane * 33 + e] = __uint_as_float(v[e]) * scale;
         __syncwarp();
@@ -240,7 +250,7 @@ __global__ void __launch_bounds__(kSThreads) scores_kernel(const __grid_constant
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int rr = 4 * i + rr0;
-          const int gr = i0 + warp * 32 + rr;
+          const int gr = i0 + quad * 32 + rr;
           if (gr < g.Nb && gj < g.Nb) {
             const float* t = tr + rr * 33 + cc;
             *reinterpret_cast<float4*>(s + (bh * g.Nb + gr) * (long long)g.Nb + gj) = make_float4(t[0], t[1], t[2], t[3]);
@@ -251,9 +261,9 @@ __global__ void __launch_bounds__(kSThreads) scores_kernel(const __grid_constant
     } else {
       float* srow = s + (bh * g.Nb + gi) * (long long)g.Nb + j0;
 #pragma unroll 1
-      for (int c = 0; c < kSTile / 32; ++c) {
+      for (int c = c0; c < c0 + kSTile / 64; ++c) {
         uint32_t v[32];
-        ptx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c * 32, v);
+        ptx::tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + c * 32, v);
         if (gi < g.Nb) {
           const int cb = c * 32;
 #pragma unroll
@@ -303,8 +313,7 @@ __device__ __forceinline__ float key_value(uint32_t k) {
 // adding 1.5 * 2^23 (the sum's low mantissa bits are the rounded value).  Each step is
 // monotone in v, so the bin never decreases as the key grows; equal keys share a bin.
 __device__ __forceinline__ int bin_index(uint32_t k, float sc, float off) {
-  const float x = fminf(fmaxf(__fmaf_rn(key_value(k), sc, off), 0.f), 63.f);
-  return __float_as_int(__fadd_rn(x, 12582912.f)) & 63;
+  return __float_as_int(__fadd_rn(__fmaf_rn(key_value(k), sc, off), 12582912.f)) & 63;
 }
 
 // Cut of a row from a 64-bin histogram of the candidate scores, linear in value between
@@ -319,16 +328,18 @@ __device__ __forceinline__ bool cut_by_histogram(const uint32_t (&key)[KPL], uin
                                                  int m, uint32_t* hist, uint32_t* list, int lane, uint32_t& thr,
                                                  int& above, int& eqc) {
   const float vmin = key_value(lo_key), vmax = key_value(hi_key);
-  const float sc = 64.f / (vmax - vmin);
+  const float sc = 63.f / (vmax - vmin);
   const float off = -vmin * sc;
-  // equal ends (one bin), or ends whose range does not give finite bin arithmetic
-  if (!(vmax > vmin) || !(sc <= 3.0e38f) || !(fabsf(off) <= 3.0e38f)) return false;
+  // Equal ends (one bin), or an offset too large for fma(v, sc, off) to stay within 1/4 of
+  // [0, 63] on [vmin, vmax] (its rounding errors are below 2 |off| 2^-24): then rounding
+  // to the nearest integer gives a bin in 0 .. 63 without clamping.
+  if (!(vmax > vmin) || !(fabsf(off) <= 1048576.f)) return false;
   reinterpret_cast<uint2*>(hist)[lane] = make_uint2(0u, 0u);
   __syncwarp();
-  int bin[KPL];
+  int bin[KPL];  // 64 for the pad and sink slots (key 0)
 #pragma unroll
   for (int k = 0; k < KPL; ++k) {
-    bin[k] = bin_index(key[k], sc, off);
+    bin[k] = key[k] != 0u ? bin_index(key[k], sc, off) : 64;
     if (key[k] != 0u) atomicAdd(&hist[bin[k]], 1u);
   }
   __syncwarp();
@@ -354,7 +365,7 @@ __device__ __forceinline__ bool cut_by_histogram(const uint32_t (&key)[KPL], uin
   int cnt = 0;
 #pragma unroll
   for (int k = 0; k < KPL; ++k) {
-    const bool in = key[k] != 0u && bin[k] == B;
+    const bool in = bin[k] == B;
     const uint32_t bal = __ballot_sync(0xffffffffu, in);
     if (in) list[cnt + __popc(bal & ((1u << lane) - 1u))] = key[k];
     cnt += __popc(bal);
@@ -382,12 +393,12 @@ __device__ __forceinline__ void topk_row(const float* __restrict__ sr, int32_t* 
                                          int32_t* __restrict__ cnt_out, int Nb, int kmax, int kept,
                                          int nsink, int lane, uint32_t* hist, uint32_t* list) {
   uint32_t key[KPL];
-  uint32_t kmin = 0xffffffffu, kmax_key = 0u;
+  uint32_t kmin1 = 0xffffffffu, kmax_key = 0u;  // kmin1: smallest key - 1 (key 0 wraps to the top)
 #pragma unroll
   for (int k = 0; k < KPL; ++k) {
     const int j = k * 32 + lane;
     key[k] = (j < Nb && j >= nsink) ? order_key(__ldg(sr + j)) : 0u;
-    if (key[k] != 0u) kmin = min(kmin, key[k]);
+    kmin1 = min(kmin1, key[k] - 1u);
     kmax_key = max(kmax_key, key[k]);
   }
   const int m = kept - nsink;
@@ -400,7 +411,7 @@ __device__ __forceinline__ void topk_row(const float* __restrict__ sr, int32_t* 
   } else if (m >= ncand) {
     thr = 1u;           // every candidate
   } else {
-    const uint32_t lo_key = __reduce_min_sync(0xffffffffu, kmin);
+    const uint32_t lo_key = __reduce_min_sync(0xffffffffu, kmin1) + 1u;
     const uint32_t hi_key = __reduce_max_sync(0xffffffffu, kmax_key);
     if (!cut_by_histogram<KPL>(key, lo_key, hi_key, m, hist, list, lane, thr, above, eqc)) {
       // Bracket [lo, hi): #{key >= lo} = c_lo >= m > c_hi = #{key >= hi}.  Each step tries
@@ -492,7 +503,7 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
   const int lane = threadIdx.x & 31;
   const int w = threadIdx.x >> 5;
   const long long row = (long long)blockIdx.x * kTopkWarps + w;
-  ptx::grid_dep_wait();  // the scores come from the scores kernel, which may still be finishing
+  grid_dep_wait();  // the scores come from the scores kernel, which may still be finishing
   if (row >= rows) return;
   topk_row<KPL>(s + row * Nb, idx + row * kmax, cnt + row, Nb, kmax, kept, nsink, lane, hist_s[w], list_s[w]);
 }
@@ -544,8 +555,12 @@ static bool make_parts_map(CUtensorMap* m, const void* base, const Geo& g) {
 
 template <int D>
 cudaError_t launch_scores_d(const __nv_bfloat16* q3, const __nv_bfloat16* k3, float* scores, const Geo& g,
-                            float scale, int32_t* status, cudaStream_t s) {
+                            float scale, int nsink, int32_t* status, cudaStream_t s) {
   using C = ScoresCfg<D>;
+  // The top-k never reads a sink column's score (the sink is always kept): columns start
+  // at the sink boundary rounded down to 32 (so that stores stay 128-byte aligned).
+  const int jbase = nsink & ~31;
+  if (jbase >= g.Nb) return cudaSuccess;  // every block is a sink block: no score is read
   CUtensorMap ta, tb;
   if (!make_parts_map(&ta, q3, g) || !make_parts_map(&tb, k3, g)) return cudaErrorInvalidValue;
   static int configured_device = -1;  // one flag per instance (per D)
@@ -556,14 +571,15 @@ cudaError_t launch_scores_d(const __nv_bfloat16* q3, const __nv_bfloat16* k3, fl
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  dim3 grid((g.Nb + kSTile - 1) / kSTile, (g.Nb + kSTile - 1) / kSTile, g.B * g.heads);
-  return launch_dependent(scores_kernel<D>, grid, dim3(kSThreads), C::kSmem, s, ta, tb, scores, g, scale, status);
+  dim3 grid((g.Nb - jbase + kSTile - 1) / kSTile, (g.Nb + kSTile - 1) / kSTile, g.B * g.heads);
+  return launch_dependent(scores_kernel<D>, grid, dim3(kSThreads), C::kSmem, s, ta, tb, scores, g, scale, jbase,
+                          status);
 }
 
 cudaError_t launch_scores(const __nv_bfloat16* q3, const __nv_bfloat16* k3, float* scores, const Geo& g,
-                          float scale, int32_t* status, cudaStream_t s) {
-  if (g.D == 128) return launch_scores_d<128>(q3, k3, scores, g, scale, status, s);
-  return launch_scores_d<64>(q3, k3, scores, g, scale, status, s);
+                          float scale, int nsink, int32_t* status, cudaStream_t s) {
+  if (g.D == 128) return launch_scores_d<128>(q3, k3, scores, g, scale, nsink, status, s);
+  return launch_scores_d<64>(q3, k3, scores, g, scale, nsink, status, s);
 }
 
 cudaError_t launch_topk(const float* scores, int32_t* idx, int32_t* cnt, int kmax, int kept,

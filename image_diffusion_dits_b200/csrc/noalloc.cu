@@ -120,7 +120,8 @@ extern "C" int rf2_predict_mask_noalloc(const void* qp, const void* kp, const rf
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), s);
   if (e == cudaSuccess) e = rf2::launch_pool(qp, kp, m.q3, m.k3, geo, (flags & RF2_RASTER) != 0, s);
   if (e == cudaSuccess)
-    e = rf2::launch_scores(m.q3, m.k3, m.scores, geo, (float)(1.0 / sqrt((double)geo.D)), status, s);
+    e = rf2::launch_scores(m.q3, m.k3, m.scores, geo, (float)(1.0 / sqrt((double)geo.D)), sink ? geo.nsink : 0,
+                           status, s);
   if (e == cudaSuccess)
     e = rf2::launch_topk(m.scores, idx, cnt, kmax, kept, sink ? geo.nsink : 0, geo, s);
   if (e != cudaSuccess) return RF2_ERR_CUDA;

@@ -346,7 +346,8 @@ static int predict_mask_impl(const void* qp, const void* kp, const Geo& geo, dou
   log_geo("predict_mask", geo, kept);
   cudaError_t e = rf2::launch_pool(qp, kp, w.m.q3, w.m.k3, geo, (flags & RF2_RASTER) != 0, s);
   if (e == cudaSuccess)
-    e = rf2::launch_scores(w.m.q3, w.m.k3, w.m.scores, geo, (float)(1.0 / sqrt((double)geo.D)), w.status, s);
+    e = rf2::launch_scores(w.m.q3, w.m.k3, w.m.scores, geo, (float)(1.0 / sqrt((double)geo.D)),
+                           nsink_of(geo, sink), w.status, s);
   if (e == cudaSuccess)
     e = rf2::launch_topk(w.m.scores, idx, cnt, kmax, kept, nsink_of(geo, sink), geo, s);
   return cuda_status(e);

@@ -180,7 +180,7 @@ cudaError_t launch_pool(const void* qp, const void* kp, __nv_bfloat16* q3, __nv_
 // Pooled scores s = qbar . kbar * scale from the bf16 parts (tcgen05); status (may be
 // null) receives RF2_ERR_TIMEOUT if a wait ran out.
 cudaError_t launch_scores(const __nv_bfloat16* q3, const __nv_bfloat16* k3, float* scores, const Geo& g,
-                          float scale, int32_t* status, cudaStream_t s);
+                          float scale, int nsink, int32_t* status, cudaStream_t s);
 cudaError_t launch_topk(const float* scores, int32_t* idx, int32_t* cnt, int kmax, int kept,
                         int nsink, const Geo& g, cudaStream_t s);
 // Returns cudaErrorNotSupported when the shape has no kernel instance.  raster: Q/K/V

@@ -124,14 +124,6 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// Programmatic dependent launch.  A kernel launched with programmatic stream
-// serialization may start while the kernel before it in the stream is finishing;
-// grid_dep_wait blocks (in hardware) until that kernel has completed and its writes are
-// visible.  grid_dep_launch lets the next such kernel be scheduled once every CTA of this
-// grid has executed it.  Both are no-ops for a kernel launched without the attribute.
-__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
