@@ -125,6 +125,20 @@ def test_predict_mask_cut_by_histogram_and_by_search(case):
             assert np.all(cnt.cpu().numpy() == sel.kept)
 
 
+@pytest.mark.parametrize("shape", [
+    # one temporal window: all 64 blocks are sink blocks, so no score is computed at all
+    dict(B=1, heads=2, T=1, H=64, W=64, D=64, wt=1, wh=8, ww=8),
+    # 32 sink blocks: the score columns start exactly at the sink boundary
+    dict(B=1, heads=2, T=3, H=32, W=64, D=64, wt=1, wh=8, ww=8),
+])
+def test_predict_mask_score_columns_from_the_sink_boundary(shape):
+    """The scores kernel computes only the columns from the sink count rounded down to 32
+    (the top-k reads no sink column's score) and is not launched when every block is a
+    sink block; the lists still equal the oracle's, with and without the sink."""
+    for s_, sink in ((0.8, True), (0.5, True), (0.8, False)):
+        _mask_case(shape, s_, sink, False, seed=1700)
+
+
 @pytest.mark.parametrize("shape", RAGGED)
 def test_permute_unpermute_ragged_bit_exact(shape):
     g, og = rf2.Geometry(**shape), O.geom(**shape)
