@@ -7,9 +7,11 @@
 //   scores : s[b, head, i, j] = qbar_i . kbar_j * scale on the tensor cores: each mean is
 //            split into three bf16 parts (hi + mid + lo, about 24 significant bits) and
 //            the six products that matter at fp32 precision are accumulated in fp32.
+//            Columns of sink blocks below a multiple of 32 are not computed.
 //   topk   : per row, the sink blocks plus the m best other blocks (ties to the lower
-//            id) as an ascending list; one warp per row, a bracketed search for the cut
-//            (interpolation and bisection steps in turn) that ends on the exact m-th key.
+//            id) as an ascending list; one warp per row, the exact m-th key found from a
+//            value histogram of the row (a bracketed search where the histogram cannot
+//            isolate it).
 #include "rf2_common.cuh"
 #include "sm100_ptx.cuh"
 
@@ -283,11 +285,12 @@ __global__ void __launch_bounds__(kSThreads) scores_kernel(const __grid_constant
 
 // ------------------------------------------------------------------------------- top-k
 // One warp per (b, head, i) row.  Scores map to order-preserving uint32 keys (every real
-// key is > 0; 0 marks a non-candidate).  The threshold is found exactly by a bracketed
-// search over the key range with warp-wide counts (interpolated and bisection steps in
-// turn), stopping as soon as exactly m candidates lie at or above it; candidates above it
-// are kept, and equal ones in ascending block order until m are kept.  The output list (sink blocks and kept candidates) is
-// emitted in ascending order with ballots.
+// key is > 0; 0 marks a non-candidate).  The threshold thr, the m-th largest candidate
+// key, is found exactly: from a 64-bin value histogram of the row (cut_by_histogram), or,
+// where that cannot isolate it, by a bracketed search over the key range with warp-wide
+// counts (interpolated and bisection steps in turn).  Candidates above thr are kept, and
+// equal ones in ascending block order until m are kept.  The output list (sink blocks,
+// then kept candidates) is emitted in ascending order with ballots.
 constexpr int kTopkWarps = 8;
 constexpr int kMaxPerLane = 32;  // Nb <= 1024
 
